@@ -1,0 +1,211 @@
+"""Sliding Tile Attention (STA) forward for NVIDIA B200 (sm_100a).
+
+A thin ctypes binding over libsta.so (include/sta.h).  PyTorch only provides
+device memory and the current CUDA stream; every step runs in the library's
+CUDA kernels.  There is no CPU fallback: if libsta.so is missing, or the
+device is not sm_100, calls raise.
+
+Method (STA README "Sliding Tile Atteniton Kernel", section Usage):
+``sliding_tile_attention(q, k, v, window_size, text_length, has_text)`` on
+[batch, heads, seq, head_dim] tensors, seq = T*H*W (+ 256 padded text
+tokens), tiles of (6, 8, 8) tokens, ``window_size`` in tiles.
+"""
+import ctypes
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+__all__ = [
+    "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
+    "forward", "sliding_tile_attention", "swa_forward", "device_status",
+    "retained_pairs", "STATUS",
+]
+
+STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
+          3: "STA_ERR_CUDA", 4: "STA_ERR_DEVICE_TIMEOUT"}
+
+EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
+            "sta_forward", "sta_forward_lse", "sta_swa_forward",
+            "sta_device_status", "sta_status_string", "sta_shutdown",
+            "sta_retained_pairs")
+
+
+class StaError(RuntimeError):
+    def __init__(self, code, where):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+_LIB = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I3 = ctypes.c_int * 3
+
+
+def lib():
+    """Loads libsta.so (built in-tree); raises if it is missing."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m block_sparse_local_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    geo = [_I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]
+    L.sta_tile_reorder.argtypes = [_P, _P] + geo + [_I, _P]
+    L.sta_tile_unreorder.argtypes = [_P, _P] + geo + [_I, _P]
+    L.sta_build_kv_tile_lists.argtypes = [_P, _P, _I, _I, _I, _I, _I,
+                                          ctypes.POINTER(ctypes.c_int),
+                                          ctypes.POINTER(ctypes.c_int), _I, _I, _P]
+    fwd = [_I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int),
+           ctypes.POINTER(ctypes.c_int), _I, _I, _P]
+    L.sta_forward.argtypes = [_P, _P, _P, _P] + fwd
+    L.sta_forward_lse.argtypes = [_P, _P, _P, _P, _P] + fwd
+    L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
+    L.sta_device_status.argtypes = [_P]
+    L.sta_status_string.argtypes = [_I]
+    L.sta_status_string.restype = ctypes.c_char_p
+    L.sta_shutdown.argtypes = []
+    L.sta_shutdown.restype = None
+    L.sta_retained_pairs.argtypes = [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int),
+                                     ctypes.POINTER(ctypes.c_int), _I, _I]
+    L.sta_retained_pairs.restype = ctypes.c_int64
+    for name in EXPORTED:
+        fn = getattr(L, name)
+        if name not in ("sta_status_string", "sta_shutdown", "sta_retained_pairs"):
+            fn.restype = ctypes.c_int
+    _LIB = L
+    return L
+
+
+def _check(code, where):
+    if code != 0:
+        raise StaError(code, where)
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _windows(window_size, heads):
+    ws = [tuple(int(x) for x in w) for w in window_size]
+    if len(ws) == 1 and heads > 1:
+        ws = ws * heads
+    if len(ws) != heads:
+        raise ValueError("window_size needs one (wt, wh, ww) per head (or one for all)")
+    arr = (ctypes.c_int * (3 * heads))(*[x for w in ws for x in w])
+    return arr
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if not t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous bf16 CUDA tensors")
+
+
+def tile_reorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
+    """[B, heads, S, d] raster order -> tile order (text rows unchanged)."""
+    _check_qkv(x)
+    out = torch.empty_like(x) if out is None else out
+    B, nh, _, d = x.shape
+    T, H, W = video_shape
+    _check(lib().sta_tile_reorder(_ptr(x), _ptr(out), B, nh, d, T, H, W, _I3(*tile),
+                                  int(has_text), _stream(x)), "sta_tile_reorder")
+    return out
+
+
+def tile_unreorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
+    """Inverse of tile_reorder."""
+    _check_qkv(x)
+    out = torch.empty_like(x) if out is None else out
+    B, nh, _, d = x.shape
+    T, H, W = video_shape
+    _check(lib().sta_tile_unreorder(_ptr(x), _ptr(out), B, nh, d, T, H, W, _I3(*tile),
+                                    int(has_text), _stream(x)), "sta_tile_unreorder")
+    return out
+
+
+def build_kv_tile_lists(window_size, video_shape, tile=(6, 8, 8), text_length=0,
+                        has_text=True, max_k=None, device="cuda"):
+    """Per-head KV tile lists: (counts [heads, NQ], ids [heads, NQ, max_k])."""
+    heads = len(window_size)
+    T, H, W = video_shape
+    NV = (T // tile[0]) * (H // tile[1]) * (W // tile[2])
+    NQ = NV + (1 if has_text else 0)
+    if max_k is None:
+        max_k = NV + 1
+    counts = torch.empty((heads, NQ), dtype=torch.int32, device=device)
+    ids = torch.empty((heads, NQ, max_k), dtype=torch.int32, device=device)
+    _check(lib().sta_build_kv_tile_lists(_ptr(counts), _ptr(ids), max_k, heads, T, H, W,
+                                         _I3(*tile), _windows(window_size, heads),
+                                         int(text_length), int(has_text), _stream(counts)),
+           "sta_build_kv_tile_lists")
+    return counts, ids
+
+
+def forward(q, k, v, window_size, text_length, has_text, video_shape,
+            tile=(6, 8, 8), out=None, return_lse=False):
+    """STA attention on TILE-ordered q, k, v [B, heads, S, d] (bf16)."""
+    _check_qkv(q, k, v)
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    out = torch.empty_like(q) if out is None else out
+    wins = _windows(window_size, nh)
+    if return_lse:
+        lse = torch.empty((B, nh, S), dtype=torch.float32, device=q.device)
+        _check(lib().sta_forward_lse(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B,
+                                     nh, d, T, H, W, _I3(*tile), wins, int(text_length),
+                                     int(has_text), _stream(q)), "sta_forward_lse")
+        return out, lse
+    _check(lib().sta_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d, T, H, W,
+                             _I3(*tile), wins, int(text_length), int(has_text),
+                             _stream(q)), "sta_forward")
+    return out
+
+
+def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
+                           video_shape=(30, 48, 80), tile=(6, 8, 8)):
+    """README-style call on RASTER-ordered q, k, v: reorder, attend, unreorder."""
+    qt = tile_reorder(q, video_shape, tile, has_text)
+    kt = tile_reorder(k, video_shape, tile, has_text)
+    vt = tile_reorder(v, video_shape, tile, has_text)
+    ot = forward(qt, kt, vt, window_size, text_length, has_text, video_shape, tile)
+    return tile_unreorder(ot, video_shape, tile, has_text)
+
+
+def swa_forward(q, k, v, window, causal=True, out=None):
+    """Token-level causal sliding-window attention, GQA: q [B,hq,S,d], k,v [B,hkv,S,d]."""
+    _check_qkv(q, k, v)
+    B, hq, S, d = q.shape
+    hkv = k.shape[1]
+    out = torch.empty_like(q) if out is None else out
+    _check(lib().sta_swa_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, hq, hkv, d, S,
+                                 int(window), int(bool(causal)), _stream(q)),
+           "sta_swa_forward")
+    return out
+
+
+def device_status(device=None):
+    """Synchronises the current stream and reports a gave-up device wait."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    s = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    _check(lib().sta_device_status(s), "sta_device_status")
+
+
+def retained_pairs(B, window_size, video_shape, tile=(6, 8, 8), text_length=0,
+                   has_text=True):
+    """Allowed (query, key) pairs of sta_forward (FLOPs = 4 * d * pairs)."""
+    heads = len(window_size)
+    T, H, W = video_shape
+    n = lib().sta_retained_pairs(B, heads, T, H, W, _I3(*tile), _windows(window_size, heads),
+                                 int(text_length), int(has_text))
+    if n < 0:
+        raise ValueError("invalid geometry")
+    return int(n)

@@ -1,0 +1,54 @@
+"""Builds libsta.so in-tree for sm_100a with nvcc.
+
+    python -m block_sparse_local_b200.build [--verbose]
+
+The library is one translation unit (csrc/sta_lib.cu includes the kernel
+headers) compiled with -gencode arch=compute_100a,code=sm_100a.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+LIB_PATH = os.path.join(HERE, "libsta.so")
+SOURCES = [os.path.join(HERE, "csrc", "sta_lib.cu")]
+DEPENDS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
+                     ("device_ptx.cuh", "reorder.cuh", "tile_lists.cuh",
+                      "attn_fwd.cuh")] + [os.path.join(ROOT, "include", "sta.h")]
+
+
+def nvcc_path():
+    cuda = os.environ.get("CUDA_HOME", "/usr/local/cuda")
+    p = os.path.join(cuda, "bin", "nvcc")
+    return p if os.path.exists(p) else "nvcc"
+
+
+def command(out=LIB_PATH, extra=()):
+    return [nvcc_path(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3",
+            "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-shared",
+            "-I" + os.path.join(ROOT, "include"), *extra, "-o", out, *SOURCES]
+
+
+def up_to_date():
+    if not os.path.exists(LIB_PATH):
+        return False
+    t = os.path.getmtime(LIB_PATH)
+    return all(os.path.getmtime(f) <= t for f in DEPENDS)
+
+
+def build(force=False, verbose=False):
+    if not force and up_to_date():
+        return LIB_PATH
+    cmd = command(extra=("-Xptxas", "-v") if verbose else ())
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if verbose or res.returncode != 0:
+        sys.stderr.write(res.stdout + res.stderr)
+    if res.returncode != 0:
+        raise RuntimeError("nvcc failed building libsta.so")
+    return LIB_PATH
+
+
+if __name__ == "__main__":
+    build(force=True, verbose="--verbose" in sys.argv)
+    print(LIB_PATH)

@@ -1,0 +1,464 @@
+// attn_fwd.cuh - fused block-sparse attention forward for sm_100a.
+//
+// Computes, for every 128-row query block, O = softmax(Q K^T / sqrt(d)) V over
+// a list of 128-key blocks, with tensor cores (tcgen05, accumulators in TMEM)
+// and an online softmax in fp32.  Two modes share the pipeline:
+//
+//  * Mode::kSta - Sliding Tile Attention (STA README, "Usage" and "Why is STA
+//    Fast?"): the key blocks of a query tile are the whole key tiles of its
+//    window, plus the padded text block.  Video tiles are always dense; only
+//    the text block, whose last columns may be padding (text_length < 256),
+//    is masked.
+//  * Mode::kSwa - token-level causal sliding-window attention with GQA (the
+//    mixed-block baseline of "Why is STA Fast?"; window over previous
+//    positions as on the sliding-window search-result page).  Blocks cut by
+//    the band edges are masked per element.
+//
+// CTA = 10 warps, one work item = up to two 128-row query blocks that read
+// the same key blocks:
+//   warp 0      TMA producer (one thread): Q once, then K and V blocks into
+//               K / V rings of shared-memory stages (128-byte swizzle).
+//   warp 1      MMA issuer (one thread) and TMEM owner:
+//               S_i = Q_i K^T (SS, M=128 N=128 K=d), O_i += P_i V (TS: P
+//               from TMEM, V from shared memory, N=d), ping-ponging the two
+//               slots so the tensor pipe works on one slot while the other
+//               slot's softmax runs.
+//   warps 2-5   softmax of slot 0, warps 6-9 softmax of slot 1: one thread
+//               per query row (TMEM lane), reads its 128 scores, updates the
+//               running max / sum, writes bf16 P over the first 64 columns
+//               of S, rescales its O row when the max grew by more than
+//               2^8, and finally normalises O and stores it.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
+// O1 [256+d, 256+2d); P_i aliases the first 64 columns of S_i.  The MMA that
+// overwrites S_i with the next scores is issued after the P_i.V MMA that
+// reads P_i; tcgen05 MMAs of one thread execute in issue order.
+#pragma once
+
+#include "device_ptx.cuh"
+
+namespace sta {
+
+constexpr int kBM = 128;        // query rows per block (MMA M)
+constexpr int kBN = 128;        // keys per block
+constexpr int kFwdThreads = 320;
+constexpr int kWarpTma = 0;
+constexpr int kWarpMma = 1;
+constexpr int kWarpSoftmax0 = 2;
+
+enum class Mode { kSta = 0, kSwa = 1 };
+
+struct WorkItem {
+  int q0;       // first row (in the [B*heads*S, d] view) of query block 0
+  int q1;       // same for block 1, or -1
+  int kv_base;  // first row of the key/value slice
+  int list;     // kSta: tile-list row; kSwa: query block index
+};
+
+struct FwdParams {
+  const WorkItem* items;
+  const int* counts;
+  const int* ids;
+  int max_k;
+  int tile_blocks;    // tile volume / 128
+  int V;              // tile volume
+  int L_v;            // video rows of a slice
+  int text_len;       // valid text keys
+  int text_blocks;    // key blocks of the text block holding valid keys
+  int text_sentinel;  // lists end with the text block
+  int window;         // kSwa: tokens
+  float scale_log2;   // log2(e) / sqrt(d)
+  __nv_bfloat16* out;
+  float* lse;
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kPanels = D / 64;          // 128-byte swizzle panels
+  static constexpr int kPanelBytes = 128 * 128;   // 128 rows x 128 bytes
+  static constexpr int kBlockBytes = kBM * D * 2;
+  static constexpr int kKStages = D == 128 ? 2 : 4;
+  static constexpr int kVStages = D == 128 ? 2 : 4;
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kQOff + 2 * kBlockBytes;
+  static constexpr int kVOff = kKOff + kKStages * kBlockBytes;
+  static constexpr int kBarOff = kVOff + kVStages * kBlockBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, align
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kOCol = 256;
+};
+
+// Key-block sequence of one work item, identical for all roles.
+struct KvSeq {
+  int n;            // number of key blocks
+  int nvid;         // kSta: video blocks before the text blocks
+  const int* ids;   // kSta: tile ids of the list
+  int kv_base;
+  int qb;           // kSwa: query block
+};
+
+template <Mode M>
+__device__ __forceinline__ KvSeq make_seq(const FwdParams& p, const WorkItem& it) {
+  KvSeq s;
+  s.kv_base = it.kv_base;
+  if constexpr (M == Mode::kSta) {
+    const int cnt = p.counts[it.list];
+    s.ids = p.ids + static_cast<size_t>(it.list) * p.max_k;
+    s.nvid = (cnt - p.text_sentinel) * p.tile_blocks;
+    s.n = s.nvid + (p.text_sentinel ? p.text_blocks : 0);
+    s.qb = 0;
+  } else {
+    s.qb = it.list;
+    int lo = s.qb * kBN - p.window + 1;     // smallest key of the band
+    int kb_lo = lo <= 0 ? 0 : lo / kBN;
+    s.n = s.qb - kb_lo + 1;                 // diagonal block first
+    s.nvid = s.n;
+    s.ids = nullptr;
+  }
+  return s;
+}
+
+template <Mode M>
+__device__ __forceinline__ int seq_row(const FwdParams& p, const KvSeq& s, int j) {
+  if constexpr (M == Mode::kSta) {
+    if (j < s.nvid) {
+      const int t = j / p.tile_blocks;
+      return s.kv_base + s.ids[t] * p.V + (j - t * p.tile_blocks) * kBN;
+    }
+    return s.kv_base + p.L_v + (j - s.nvid) * kBN;
+  } else {
+    return s.kv_base + (s.qb - j) * kBN;
+  }
+}
+
+// Valid column range [lo, hi) of block j for query row r, or false when the
+// block needs no mask.
+template <Mode M>
+__device__ __forceinline__ bool seq_mask(const FwdParams& p, const KvSeq& s, int j,
+                                         int r, int& lo, int& hi) {
+  if constexpr (M == Mode::kSta) {
+    if (j < s.nvid) return false;
+    const int col0 = (j - s.nvid) * kBN;
+    if (col0 + kBN <= p.text_len) return false;
+    lo = 0;
+    hi = p.text_len - col0;
+    return true;
+  } else {
+    const int kb = s.qb - j;
+    const bool edge = kb * kBN < s.qb * kBN + (kBN - 1) - p.window + 1;
+    if (kb != s.qb && !edge) return false;
+    const int qi = s.qb * kBN + r;                 // query position
+    const int first = qi - p.window + 1 - kb * kBN;  // lowest allowed column
+    const int last = qi - kb * kBN;                // highest allowed column
+    lo = first < 0 ? 0 : first;
+    hi = last + 1 > kBN ? kBN : last + 1;
+    return true;
+  }
+}
+
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(a, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer_ns() - t0 > 200000000ull) {
+      raise_error(1u);
+      return false;
+    }
+  }
+}
+
+template <int D, Mode M>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const FwdParams p) {
+  using C = FwdCfg<D>;
+  constexpr int KST = C::kKStages;
+  constexpr int VST = C::kVStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + KST;
+  uint64_t* v_full = k_empty + KST;
+  uint64_t* v_empty = v_full + VST;
+  uint64_t* s_full = v_empty + VST;   // [2]
+  uint64_t* p_full = s_full + 2;      // [2]
+  uint64_t* o_full = p_full + 2;      // [2]
+  uint64_t* mma_done = o_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WorkItem item = p.items[blockIdx.x];
+  const bool two = item.q1 >= 0;
+  const KvSeq seq = make_seq<M>(p, item);
+  const int n = seq.n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    for (int i = 0; i < VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&o_full[i], 1);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpTma && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  if (warp == kWarpMma) tmem_alloc(tmem_holder, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const bool skip = *abort_flag != 0;
+
+  const uint32_t smem_q = smem_u32(smem + C::kQOff);
+  const uint32_t smem_k = smem_u32(smem + C::kKOff);
+  const uint32_t smem_v = smem_u32(smem + C::kVOff);
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !skip) {
+      const uint64_t pol_kv = policy_evict_last();
+      mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
+      for (int s = 0; s < (two ? 2 : 1); ++s) {
+        const int qrow = s ? item.q1 : item.q0;
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d(smem + C::kQOff + s * C::kBlockBytes + pn * C::kPanelBytes,
+                      &tmap_q, q_full, pn * 64, qrow);
+      }
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int ks = j % KST;
+        if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, abort_flag)) break;
+        const int row = seq_row<M>(p, seq, j);
+        mbar_arrive_expect_tx(&k_full[ks], C::kBlockBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d_hint(smem + C::kKOff + ks * C::kBlockBytes + pn * C::kPanelBytes,
+                           &tmap_k, &k_full[ks], pn * 64, row, pol_kv);
+        const int vs = j % VST;
+        if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, abort_flag)) {
+          issued = j * 2 + 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[vs], C::kBlockBytes);
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn)
+          tma_load_2d_hint(smem + C::kVOff + vs * C::kBlockBytes + pn * C::kPanelBytes,
+                           &tmap_v, &v_full[vs], pn * 64, row, pol_kv);
+        issued = j * 2 + 2;
+      }
+      // Leave no copy in flight: wait for the last load of every stage.
+      mbar_wait_drain(q_full, 0);
+      const int nk = (issued + 1) / 2, nv = issued / 2;
+      for (int s = 0; s < KST && s < nk; ++s) {
+        const int last = s + ((nk - 1 - s) / KST) * KST;
+        mbar_wait_drain(&k_full[s], (last / KST) & 1);
+      }
+      for (int s = 0; s < VST && s < nv; ++s) {
+        const int last = s + ((nv - 1 - s) / VST) * VST;
+        mbar_wait_drain(&v_full[s], (last / VST) & 1);
+      }
+    }
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !skip) {
+      constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false);
+      constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, true);
+      auto t_s = [&](int slot) { return tmem + (slot ? 128u : 0u); };
+      auto t_o = [&](int slot) { return tmem + C::kOCol + (slot ? uint32_t(D) : 0u); };
+      auto issue_s = [&](int slot, int ks) {
+        const uint32_t qa = smem_q + slot * C::kBlockBytes;
+        const uint32_t ka = smem_k + ks * C::kBlockBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          umma_ss(t_s(slot), sdesc_sw128(qa + off, 16, 1024),
+                  sdesc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int slot, int vs, bool acc) {
+        const uint32_t va = smem_v + vs * C::kBlockBytes;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          umma_ts(t_o(slot), t_s(slot) + kk * 8,
+                  sdesc_sw128(va + kk * 16 * 128, C::kPanelBytes, 1024), kIdescPV,
+                  (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        umma_commit(&s_full[0]);
+        if (two) {
+          issue_s(1, 0);
+          umma_commit(&s_full[1]);
+        }
+        umma_commit(&k_empty[0]);
+        for (int j = 0; j < n; ++j) {
+          const int vs = j % VST;
+          const int jn = j + 1;
+          const int ksn = jn % KST;
+          if (!mbar_wait(&p_full[0], j & 1, abort_flag)) break;
+          if (!mbar_wait(&v_full[vs], (j / VST) & 1, abort_flag)) break;
+          tc_fence_after();
+          issue_pv(0, vs, j > 0);
+          if (jn < n) {
+            if (!mbar_wait(&k_full[ksn], (jn / KST) & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_s(0, ksn);
+            umma_commit(&s_full[0]);
+          } else {
+            umma_commit(&o_full[0]);
+          }
+          if (two) {
+            if (!mbar_wait(&p_full[1], j & 1, abort_flag)) break;
+            tc_fence_after();
+            issue_pv(1, vs, j > 0);
+            if (jn < n) {
+              issue_s(1, ksn);
+              umma_commit(&s_full[1]);
+            } else {
+              umma_commit(&o_full[1]);
+            }
+          }
+          umma_commit(&v_empty[vs]);
+          if (jn < n) umma_commit(&k_empty[ksn]);
+        }
+      }
+      // No MMA may still run when TMEM is released.
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int slot = (warp - kWarpSoftmax0) >> 2;
+    const int sub = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = sub * 32 + lane;            // query row inside the block
+    if (!skip && (slot == 0 || two)) {
+      const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u);
+      const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0);
+      const float sl2 = p.scale_log2;
+      float m_run = -INFINITY;   // running max, log2 units of the scaled scores
+      float l_run = 0.f;
+      bool done = true;
+      for (int j = 0; j < n; ++j) {
+        if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        uint32_t sr[128];
+        STA_TMEM_LD32(t_s + 0, (sr + 0));
+        STA_TMEM_LD32(t_s + 32, (sr + 32));
+        STA_TMEM_LD32(t_s + 64, (sr + 64));
+        STA_TMEM_LD32(t_s + 96, (sr + 96));
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        int lo, hi;
+        if (seq_mask<M>(p, seq, j, r, lo, hi)) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c < lo || c >= hi) s[c] = -INFINITY;
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float m_cand = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        const bool resc = m_cand > m_run + 8.0f;
+        float alpha = 1.f;
+        if (resc) {
+          alpha = fast_exp2(m_run - m_cand);
+          m_run = m_cand;
+          l_run *= alpha;
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
+            const float p1 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
+            ls0 += p0;
+            ls1 += p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          STA_TMEM_ST16(t_s + cc * 16, pk);
+        }
+        l_run += ls0 + ls1;
+        if (j > 0 && __any_sync(0xffffffffu, resc)) {
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            STA_TMEM_LD32(t_o + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            STA_TMEM_ST32(t_o + cc * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[slot]);
+      }
+      if (done && mbar_wait_warp(&o_full[slot], 0, abort_flag)) {
+        tc_fence_after();
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const int qrow = (slot ? item.q1 : item.q0) + r;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(qrow) * D);
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          STA_TMEM_LD32(t_o + cc * 32, o);
+          tmem_wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                __uint_as_float(o[2 * e + 1]) * inv);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                          pk[4 * v4 + 3]);
+        }
+        if (p.lse != nullptr) {
+          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+          p.lse[qrow] = (m_use + __log2f(l_run)) * 0.69314718055994531f;
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace sta

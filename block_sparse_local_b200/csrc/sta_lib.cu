@@ -1,0 +1,647 @@
+// sta_lib.cu - host side of libsta.so: argument checks, planning, TMA
+// descriptors, workspace and launches behind the C ABI of include/sta.h.
+//
+// One translation unit: the kernels are included from the .cuh files so the
+// device error word has a single definition.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "sta.h"
+#include "device_ptx.cuh"
+#include "reorder.cuh"
+#include "tile_lists.cuh"
+#include "attn_fwd.cuh"
+
+namespace {
+
+using sta::FwdParams;
+using sta::Mode;
+using sta::WorkItem;
+
+constexpr int kMaxClasses = sta::kMaxWindowClasses;
+
+#define STA_CUDA_TRY(expr)                         \
+  do {                                             \
+    cudaError_t e_ = (expr);                       \
+    if (e_ != cudaSuccess) return STA_ERR_CUDA;    \
+  } while (0)
+
+// ------------------------------------------------------------------ device
+struct DeviceInfo {
+  bool checked = false;
+  bool sm100 = false;
+  int num_sms = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+sta_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= 64) return STA_ERR_CUDA;
+  DeviceInfo& di = g_dev[*dev];
+  if (!di.checked) {
+    int major = 0, minor = 0, sms = 0;
+    STA_CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev));
+    STA_CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev));
+    STA_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev));
+    di.sm100 = (major == 10 && minor == 0);
+    di.num_sms = sms;
+    di.checked = true;
+  }
+  return STA_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// [rows, d] bf16 row-major, box of 128 rows x 64 columns, 128-byte swizzle.
+sta_status make_row_map(CUtensorMap* map, const void* base, int64_t rows, int d) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return STA_ERR_CUDA;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 128};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? STA_OK : STA_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------ geometry
+struct Geom {
+  int T, H, W, ct, ch, cw;
+  int NT, NH, NW, NV, V, Lv, S;
+  bool has_text;
+  int text_len;
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sta_status make_geom(Geom* g, int T, int H, int W, const int tile[3], int has_text,
+                     int text_len) {
+  if (tile == nullptr) return STA_ERR_INVALID_ARG;
+  if (T < 1 || H < 1 || W < 1) return STA_ERR_INVALID_ARG;
+  if (tile[0] < 1 || tile[1] < 1 || tile[2] < 1) return STA_ERR_INVALID_ARG;
+  if (T % tile[0] || H % tile[1] || W % tile[2]) return STA_ERR_INVALID_ARG;
+  if (has_text != 0 && has_text != 1) return STA_ERR_INVALID_ARG;
+  const int64_t lv = static_cast<int64_t>(T) * H * W;
+  if (lv + STA_TEXT_PAD > (int64_t(1) << 30)) return STA_ERR_INVALID_ARG;
+  g->T = T; g->H = H; g->W = W;
+  g->ct = tile[0]; g->ch = tile[1]; g->cw = tile[2];
+  g->NT = T / tile[0]; g->NH = H / tile[1]; g->NW = W / tile[2];
+  g->NV = g->NT * g->NH * g->NW;
+  g->V = tile[0] * tile[1] * tile[2];
+  g->Lv = static_cast<int>(lv);
+  g->has_text = has_text != 0;
+  g->S = g->Lv + (g->has_text ? STA_TEXT_PAD : 0);
+  g->text_len = g->has_text ? text_len : 0;
+  if (g->has_text && (text_len < 0 || text_len > STA_TEXT_PAD)) return STA_ERR_INVALID_ARG;
+  return STA_OK;
+}
+
+void window_range_host(int c, int w, int n, int* s, int* e) {
+  *e = std::min(w, n);
+  *s = c - *e / 2;
+  if (*s < 0) *s = 0;
+  if (*s > n - *e) *s = n - *e;
+}
+
+sta_status check_windows(const int* window, int heads) {
+  if (window == nullptr) return STA_ERR_INVALID_ARG;
+  for (int h = 0; h < heads; ++h)
+    for (int a = 0; a < 3; ++a)
+      if (window[3 * h + a] < 1) return STA_ERR_INVALID_ARG;
+  return STA_OK;
+}
+
+// Window classes: distinct windows, heads mapped onto them in first-seen order.
+struct Classes {
+  std::vector<int> head_class;
+  std::vector<int> win;   // [nclass][3]
+  int nclass = 0;
+};
+
+Classes make_classes(const int* window, int heads) {
+  Classes c;
+  c.head_class.resize(heads);
+  for (int h = 0; h < heads; ++h) {
+    int found = -1;
+    for (int k = 0; k < c.nclass; ++k)
+      if (c.win[3 * k] == window[3 * h] && c.win[3 * k + 1] == window[3 * h + 1] &&
+          c.win[3 * k + 2] == window[3 * h + 2]) {
+        found = k;
+        break;
+      }
+    if (found < 0) {
+      found = c.nclass++;
+      c.win.insert(c.win.end(), {window[3 * h], window[3 * h + 1], window[3 * h + 2]});
+    }
+    c.head_class[h] = found;
+  }
+  return c;
+}
+
+int class_video_tiles(const Geom& g, const int* w) {
+  return std::min(w[0], g.NT) * std::min(w[1], g.NH) * std::min(w[2], g.NW);
+}
+
+void launch_lists(int* counts, int* ids, const Classes& cls, const Geom& g, int max_k,
+                  cudaStream_t st) {
+  sta::ListWindows wp;
+  std::memset(&wp, 0, sizeof(wp));
+  std::memcpy(wp.w, cls.win.data(), sizeof(int) * cls.win.size());
+  sta::ListGeom lg;
+  lg.NT = g.NT; lg.NH = g.NH; lg.NW = g.NW; lg.NV = g.NV;
+  lg.NQ = g.NV + (g.has_text ? 1 : 0);
+  lg.max_k = max_k;
+  lg.text_block = (g.has_text && g.text_len > 0) ? 1 : 0;
+  const int total = cls.nclass * lg.NQ;
+  const int threads = 128;
+  sta::kv_tile_list_kernel<<<(total + threads - 1) / threads, threads, 0, st>>>(
+      counts, ids, wp, cls.nclass, lg);
+}
+
+// ------------------------------------------------------------------ workspace
+struct Workspace {
+  void* buf = nullptr;
+  size_t cap = 0;
+  std::string plan_key;     // key of the plan currently resident in `buf`
+  std::vector<WorkItem> items;
+};
+Workspace g_ws[64];
+
+sta_status ensure_workspace(int dev, size_t bytes) {
+  Workspace& w = g_ws[dev];
+  if (w.cap >= bytes) return STA_OK;
+  if (w.buf != nullptr) {
+    STA_CUDA_TRY(cudaFree(w.buf));
+    w.buf = nullptr;
+    w.cap = 0;
+  }
+  size_t cap = std::max<size_t>(bytes, size_t(1) << 20);
+  STA_CUDA_TRY(cudaMalloc(&w.buf, cap));
+  w.cap = cap;
+  w.plan_key.clear();
+  return STA_OK;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ------------------------------------------------------------------ STA plan
+// Work items pair two 128-row query blocks with the same key-tile list so
+// both slots of a CTA share every K/V load.  Blocks of one tile pair up;
+// with an odd number of blocks per tile the leftover blocks of tiles whose
+// windows start at the same tile (hence have identical lists) pair up; the
+// text query block (256 rows) is one pair.  Items are ordered longest first
+// (text items, then by list length) and, within one length, by slice so that
+// concurrently running CTAs share K/V in L2.
+std::vector<WorkItem> plan_sta(const Geom& g, const Classes& cls, int B, int heads,
+                               int max_k, std::vector<int>* lengths) {
+  const int NQ = g.NV + (g.has_text ? 1 : 0);
+  const int bpt = g.V / sta::kBM;
+  const int text_blocks = (g.text_len + sta::kBN - 1) / sta::kBN;
+  const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
+  struct Entry { int len; int slice; WorkItem it; };
+  std::vector<Entry> all;
+  for (int b = 0; b < B; ++b) {
+    for (int h = 0; h < heads; ++h) {
+      const int slice = b * heads + h;
+      const int base = slice * g.S;
+      const int c = cls.head_class[h];
+      const int* w = &cls.win[3 * c];
+      const int vlen = class_video_tiles(g, w) * bpt + sentinel * text_blocks;
+      std::map<int64_t, int> pending;   // start triple -> leftover block row
+      for (int t = 0; t < g.NV; ++t) {
+        const int list = c * NQ + t;
+        const int row0 = base + t * g.V;
+        int qb = 0;
+        for (; qb + 1 < bpt; qb += 2)
+          all.push_back({vlen, slice, {row0 + qb * sta::kBM, row0 + (qb + 1) * sta::kBM, base, list}});
+        if (qb < bpt) {
+          const int qw = t % g.NW, qh = (t / g.NW) % g.NH, qt = t / (g.NW * g.NH);
+          int st, sh, sw, e;
+          window_range_host(qt, w[0], g.NT, &st, &e);
+          window_range_host(qh, w[1], g.NH, &sh, &e);
+          window_range_host(qw, w[2], g.NW, &sw, &e);
+          const int64_t key = (int64_t(st) * g.NH + sh) * g.NW + sw;
+          auto itp = pending.find(key);
+          if (itp == pending.end()) {
+            pending[key] = t;
+          } else {
+            const int t0 = itp->second;
+            pending.erase(itp);
+            all.push_back({vlen, slice,
+                           {base + t0 * g.V + qb * sta::kBM, row0 + qb * sta::kBM, base,
+                            c * NQ + t0}});
+          }
+        }
+      }
+      for (auto& kv : pending) {
+        const int t0 = kv.second;
+        all.push_back({vlen, slice, {base + t0 * g.V + (bpt - 1) * sta::kBM, -1, base, c * NQ + t0}});
+      }
+      if (g.has_text) {
+        const int tlen = g.NV * bpt + sentinel * text_blocks;
+        all.push_back({tlen, slice, {base + g.Lv, base + g.Lv + sta::kBM, base, c * NQ + g.NV}});
+      }
+    }
+  }
+  std::stable_sort(all.begin(), all.end(), [](const Entry& a, const Entry& b) {
+    if (a.len != b.len) return a.len > b.len;
+    return a.slice < b.slice;
+  });
+  std::vector<WorkItem> items;
+  items.reserve(all.size());
+  if (lengths) lengths->clear();
+  for (auto& e : all) {
+    items.push_back(e.it);
+    if (lengths) lengths->push_back(e.len);
+  }
+  (void)max_k;
+  return items;
+}
+
+std::string sta_key(int dev, int B, int heads, int d, const Geom& g, const int* window) {
+  std::string k = "sta:" + std::to_string(dev) + ":" + std::to_string(B) + ":" +
+                  std::to_string(heads) + ":" + std::to_string(d) + ":" + std::to_string(g.T) +
+                  "," + std::to_string(g.H) + "," + std::to_string(g.W) + ":" +
+                  std::to_string(g.ct) + "," + std::to_string(g.ch) + "," +
+                  std::to_string(g.cw) + ":" + std::to_string(g.has_text) + ":" +
+                  std::to_string(g.text_len) + ":";
+  for (int i = 0; i < 3 * heads; ++i) k += std::to_string(window[i]) + ",";
+  return k;
+}
+
+template <int D, Mode M>
+sta_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const FwdParams& prm, int num_items, cudaStream_t st) {
+  constexpr int smem = sta::FwdCfg<D>::kSmemBytes;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  STA_CUDA_TRY(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_fwd_kernel<D, M>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set[dev] = true;
+  }
+  sta::attn_fwd_kernel<D, M><<<num_items, sta::kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status forward_impl(const void* q, const void* k, const void* v, void* out, float* lse,
+                        int B, int heads, int d, int T, int H, int W, const int tile[3],
+                        const int* window, int text_len, int has_text, void* stream) {
+  if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return STA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1) return STA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return STA_ERR_INVALID_ARG;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, text_len);
+  if (s != STA_OK) return s;
+  s = check_windows(window, heads);
+  if (s != STA_OK) return s;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  if (g.V % sta::kBM != 0) return STA_ERR_UNSUPPORTED;
+  const int64_t total_rows = int64_t(B) * heads * g.S;
+  if (total_rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Classes cls = make_classes(window, heads);
+  if (cls.nclass > kMaxClasses) return STA_ERR_UNSUPPORTED;
+  const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
+  int max_k = 1;
+  for (int c = 0; c < cls.nclass; ++c)
+    max_k = std::max(max_k, class_video_tiles(g, &cls.win[3 * c]) + sentinel);
+  if (g.has_text) max_k = std::max(max_k, g.NV + sentinel);
+  const int NQ = g.NV + (g.has_text ? 1 : 0);
+  const size_t counts_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
+  const size_t ids_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
+
+  const std::string key = sta_key(dev, B, heads, d, g, window);
+  Workspace& ws = g_ws[dev];
+  std::vector<WorkItem> fresh;
+  const bool cached = (ws.plan_key == key && ws.buf != nullptr);
+  if (!cached) fresh = plan_sta(g, cls, B, heads, max_k, nullptr);
+  const std::vector<WorkItem>& items = cached ? ws.items : fresh;
+  const size_t items_bytes = sizeof(WorkItem) * items.size();
+  s = ensure_workspace(dev, counts_bytes + ids_bytes + items_bytes);
+  if (s != STA_OK) return s;
+  uint8_t* wbuf = static_cast<uint8_t*>(ws.buf);
+  int* d_counts = reinterpret_cast<int*>(wbuf);
+  int* d_ids = reinterpret_cast<int*>(wbuf + counts_bytes);
+  WorkItem* d_items = reinterpret_cast<WorkItem*>(wbuf + counts_bytes + ids_bytes);
+  if (ws.plan_key != key) {
+    ws.items = std::move(fresh);
+    STA_CUDA_TRY(cudaMemcpyAsync(d_items, ws.items.data(), sizeof(WorkItem) * ws.items.size(),
+                                 cudaMemcpyHostToDevice, st));
+    ws.plan_key = key;
+  }
+  const int num_items = static_cast<int>(ws.items.size());
+
+  CUtensorMap mq, mk, mv;
+  s = make_row_map(&mq, q, total_rows, d);
+  if (s == STA_OK) s = make_row_map(&mk, k, total_rows, d);
+  if (s == STA_OK) s = make_row_map(&mv, v, total_rows, d);
+  if (s != STA_OK) return s;
+
+  // a2: tile lists, rebuilt on every call.
+  launch_lists(d_counts, d_ids, cls, g, max_k, st);
+  STA_CUDA_TRY(cudaGetLastError());
+
+  FwdParams prm;
+  prm.items = d_items;
+  prm.counts = d_counts;
+  prm.ids = d_ids;
+  prm.max_k = max_k;
+  prm.tile_blocks = g.V / sta::kBM;
+  prm.V = g.V;
+  prm.L_v = g.Lv;
+  prm.text_len = g.text_len;
+  prm.text_blocks = (g.text_len + sta::kBN - 1) / sta::kBN;
+  prm.text_sentinel = sentinel;
+  prm.window = 0;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+  return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+}
+
+template <int kVec>
+void launch_permute(const void* in, void* out, const sta::ReorderGeom& rg, int slices,
+                    int to_tile, cudaStream_t st) {
+  dim3 grid(rg.num_tiles + (rg.S > rg.Lv ? 1 : 0), slices);
+  sta::tile_permute_kernel<kVec><<<grid, 256, 0, st>>>(
+      static_cast<const uint4*>(in), static_cast<uint4*>(out), rg, to_tile);
+}
+
+sta_status permute_impl(const void* in, void* out, int B, int heads, int d, int T, int H,
+                        int W, const int tile[3], int has_text, void* stream, int to_tile) {
+  if (!in || !out || in == out) return STA_ERR_INVALID_ARG;
+  if (!aligned16(in) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1 || d < 1) return STA_ERR_INVALID_ARG;
+  if (B * static_cast<int64_t>(heads) > 65535) return STA_ERR_INVALID_ARG;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, 0);
+  if (s != STA_OK) return s;
+  const int vec = d * 2 / 16;
+  if ((d * 2) % 16 != 0) return STA_ERR_UNSUPPORTED;
+  if (vec != 4 && vec != 8 && vec != 16 && vec != 32) return STA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(g.V) * vec >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  sta::ReorderGeom rg;
+  rg.T = g.T; rg.H = g.H; rg.W = g.W;
+  rg.ct = g.ct; rg.ch = g.ch; rg.cw = g.cw;
+  rg.NH = g.NH; rg.NW = g.NW;
+  rg.V = g.V; rg.S = g.S; rg.Lv = g.Lv; rg.num_tiles = g.NV;
+  rg.div_cw = sta::make_fastdiv(g.cw);
+  rg.div_chcw = sta::make_fastdiv(g.ch * g.cw);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int slices = B * heads;
+  switch (vec) {
+    case 4: launch_permute<4>(in, out, rg, slices, to_tile, st); break;
+    case 8: launch_permute<8>(in, out, rg, slices, to_tile, st); break;
+    case 16: launch_permute<16>(in, out, rg, slices, to_tile, st); break;
+    default: launch_permute<32>(in, out, rg, slices, to_tile, st); break;
+  }
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+// ------------------------------------------------------------------ SWA plan
+std::vector<WorkItem> plan_swa(int B, int hq, int hkv, int S, int window) {
+  const int group = hq / hkv;
+  const int nqb = S / sta::kBM;
+  struct Entry { int len; int kvs; WorkItem it; };
+  std::vector<Entry> all;
+  for (int b = 0; b < B; ++b)
+    for (int hk = 0; hk < hkv; ++hk) {
+      const int kv_base = (b * hkv + hk) * S;
+      for (int qb = 0; qb < nqb; ++qb) {
+        const int lo = qb * sta::kBN - window + 1;
+        const int kb_lo = lo <= 0 ? 0 : lo / sta::kBN;
+        const int len = qb - kb_lo + 1;
+        for (int g0 = 0; g0 < group; g0 += 2) {
+          const int h0 = hk * group + g0;
+          const int q0 = (b * hq + h0) * S + qb * sta::kBM;
+          const int q1 = (g0 + 1 < group) ? (b * hq + h0 + 1) * S + qb * sta::kBM : -1;
+          all.push_back({len, b * hkv + hk, {q0, q1, kv_base, qb}});
+        }
+      }
+    }
+  std::stable_sort(all.begin(), all.end(), [](const Entry& a, const Entry& b) {
+    if (a.len != b.len) return a.len > b.len;
+    return a.kvs < b.kvs;
+  });
+  std::vector<WorkItem> items;
+  for (auto& e : all) items.push_back(e.it);
+  return items;
+}
+
+}  // namespace
+
+// ====================================================================== C ABI
+extern "C" {
+
+const char* sta_status_string(sta_status s) {
+  switch (s) {
+    case STA_OK: return "STA_OK";
+    case STA_ERR_INVALID_ARG: return "STA_ERR_INVALID_ARG: argument rejected";
+    case STA_ERR_UNSUPPORTED: return "STA_ERR_UNSUPPORTED: shape or device not supported";
+    case STA_ERR_CUDA: return "STA_ERR_CUDA: a CUDA call failed";
+    case STA_ERR_DEVICE_TIMEOUT: return "STA_ERR_DEVICE_TIMEOUT: a device wait gave up";
+  }
+  return "STA_ERR_UNKNOWN";
+}
+
+sta_status sta_tile_reorder(const void* in, void* out, int B, int heads, int d, int T, int H,
+                            int W, const int tile[3], int has_text, void* stream) {
+  return permute_impl(in, out, B, heads, d, T, H, W, tile, has_text, stream, 1);
+}
+
+sta_status sta_tile_unreorder(const void* in, void* out, int B, int heads, int d, int T,
+                              int H, int W, const int tile[3], int has_text, void* stream) {
+  return permute_impl(in, out, B, heads, d, T, H, W, tile, has_text, stream, 0);
+}
+
+sta_status sta_build_kv_tile_lists(int* counts, int* ids, int max_k, int heads, int T, int H,
+                                   int W, const int tile[3], const int* window, int text_len,
+                                   int has_text, void* stream) {
+  if (!counts || !ids || heads < 1 || heads > kMaxClasses) return STA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(counts) & 3u) || (reinterpret_cast<uintptr_t>(ids) & 3u))
+    return STA_ERR_INVALID_ARG;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, text_len);
+  if (s != STA_OK) return s;
+  s = check_windows(window, heads);
+  if (s != STA_OK) return s;
+  const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
+  int need = 1;
+  for (int h = 0; h < heads; ++h)
+    need = std::max(need, class_video_tiles(g, &window[3 * h]) + sentinel);
+  if (g.has_text) need = std::max(need, g.NV + sentinel);
+  if (max_k < need) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  // one class per head: the public lists are per head
+  Classes cls;
+  cls.nclass = heads;
+  cls.win.assign(window, window + 3 * heads);
+  cls.head_class.resize(heads);
+  for (int h = 0; h < heads; ++h) cls.head_class[h] = h;
+  launch_lists(counts, ids, cls, g, max_k, reinterpret_cast<cudaStream_t>(stream));
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status sta_forward(const void* q, const void* k, const void* v, void* out, int B,
+                       int heads, int d, int T, int H, int W, const int tile[3],
+                       const int* window, int text_len, int has_text, void* stream) {
+  return forward_impl(q, k, v, out, nullptr, B, heads, d, T, H, W, tile, window, text_len,
+                      has_text, stream);
+}
+
+sta_status sta_forward_lse(const void* q, const void* k, const void* v, void* out, float* lse,
+                           int B, int heads, int d, int T, int H, int W, const int tile[3],
+                           const int* window, int text_len, int has_text, void* stream) {
+  if (lse == nullptr) return STA_ERR_INVALID_ARG;
+  return forward_impl(q, k, v, out, lse, B, heads, d, T, H, W, tile, window, text_len,
+                      has_text, stream);
+}
+
+sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* out, int B,
+                           int hq, int hkv, int d, int S, int window, int causal,
+                           void* stream) {
+  if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return STA_ERR_INVALID_ARG;
+  if (B < 1 || hq < 1 || hkv < 1 || hq % hkv != 0 || S < 1 || window < 1) return STA_ERR_INVALID_ARG;
+  if (causal != 1) return STA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  if (S % sta::kBM != 0) return STA_ERR_UNSUPPORTED;
+  const int64_t qrows = int64_t(B) * hq * S;
+  if (qrows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  sta_status s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const std::string key = "swa:" + std::to_string(dev) + ":" + std::to_string(B) + ":" +
+                          std::to_string(hq) + ":" + std::to_string(hkv) + ":" +
+                          std::to_string(S) + ":" + std::to_string(window);
+  Workspace& ws = g_ws[dev];
+  std::vector<WorkItem> fresh;
+  const bool cached = (ws.plan_key == key && ws.buf != nullptr);
+  if (!cached) fresh = plan_swa(B, hq, hkv, S, window);
+  const size_t bytes = sizeof(WorkItem) * (cached ? ws.items.size() : fresh.size());
+  s = ensure_workspace(dev, bytes);
+  if (s != STA_OK) return s;
+  WorkItem* d_items = static_cast<WorkItem*>(ws.buf);
+  if (ws.plan_key != key) {
+    ws.items = std::move(fresh);
+    STA_CUDA_TRY(cudaMemcpyAsync(d_items, ws.items.data(), sizeof(WorkItem) * ws.items.size(),
+                                 cudaMemcpyHostToDevice, st));
+    ws.plan_key = key;
+  }
+  CUtensorMap mq, mk, mv;
+  s = make_row_map(&mq, q, qrows, d);
+  if (s == STA_OK) s = make_row_map(&mk, k, int64_t(B) * hkv * S, d);
+  if (s == STA_OK) s = make_row_map(&mv, v, int64_t(B) * hkv * S, d);
+  if (s != STA_OK) return s;
+  FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.items = d_items;
+  prm.window = window;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = nullptr;
+  const int num_items = static_cast<int>(ws.items.size());
+  if (d == 128) return launch_attn<128, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
+  return launch_attn<64, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
+}
+
+sta_status sta_device_status(void* stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return STA_ERR_CUDA;
+  unsigned int word = 0;
+  STA_CUDA_TRY(cudaMemcpyFromSymbol(&word, sta::g_error_word, sizeof(word)));
+  if (word != 0) {
+    const unsigned int zero = 0;
+    STA_CUDA_TRY(cudaMemcpyToSymbol(sta::g_error_word, &zero, sizeof(zero)));
+    return STA_ERR_DEVICE_TIMEOUT;
+  }
+  if (cudaGetLastError() != cudaSuccess) return STA_ERR_CUDA;
+  return STA_OK;
+}
+
+void sta_shutdown(void) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return;
+  for (int i = 0; i < 64; ++i) {
+    if (g_ws[i].buf != nullptr) {
+      cudaSetDevice(i);
+      cudaFree(g_ws[i].buf);
+      g_ws[i] = Workspace();
+    }
+  }
+  cudaSetDevice(dev);
+}
+
+int64_t sta_retained_pairs(int B, int heads, int T, int H, int W, const int tile[3],
+                           const int* window, int text_len, int has_text) {
+  Geom g;
+  if (make_geom(&g, T, H, W, tile, has_text, text_len) != STA_OK) return -1;
+  if (B < 1 || heads < 1 || check_windows(window, heads) != STA_OK) return -1;
+  int64_t total = 0;
+  for (int h = 0; h < heads; ++h) {
+    const int64_t vid = class_video_tiles(g, &window[3 * h]);
+    int64_t per = int64_t(g.NV) * g.V * (vid * g.V + (g.has_text ? g.text_len : 0));
+    if (g.has_text) per += int64_t(STA_TEXT_PAD) * (g.Lv + g.text_len);
+    total += per;
+  }
+  return total * B;
+}
+
+}  // extern "C"

@@ -1,0 +1,148 @@
+/*
+ * sta.h - C ABI of libsta.so: Sliding Tile Attention (STA) forward on B200.
+ *
+ * Method: the STA README ("Sliding Tile Atteniton Kernel", FastVideo
+ * sta_kernel/thunderkitten), sections "Usage", "How Does STA Work?" and
+ * "Why is STA Fast?".  A (T,H,W) video token grid is cut into tiles of
+ * (ct,ch,cw) tokens ("a tile is a cube of size (6, 8, 8)"); every query tile
+ * attends to the whole key tiles inside a window of (wt,wh,ww) tiles
+ * ("window_size in tiles"), centred on the query tile and shifted inward at
+ * the grid border so it always spans the full window; 256 padded text tokens
+ * may follow the video ("text tokens = 256 with padding", text_length 0..256).
+ * Video queries also attend to the first text_len text keys; text queries
+ * attend to every video key and the first text_len text keys.  The attention
+ * map is therefore made of fully dense or fully empty tile blocks.
+ *
+ * Conventions for every entry point:
+ *  - Tensors are caller-owned device memory, bf16, contiguous
+ *    [B, heads, S, d] with S = T*H*W + (has_text ? 256 : 0), base pointers
+ *    16-byte aligned.  Nothing is freed or retained by the library.
+ *  - `stream` is a cudaStream_t passed as void*; all work is enqueued on it,
+ *    asynchronously, with no implicit synchronisation.  NULL = legacy stream.
+ *  - Arguments are checked on the host before any launch; on an error status
+ *    nothing has been enqueued and no output byte has been written.
+ *  - `tile` and `window` are HOST pointers to int32 triples.
+ *  - Outputs must not alias inputs.
+ *  - Device-side waits are bounded: a kernel that gives up records
+ *    STA_ERR_DEVICE_TIMEOUT in a device flag, read by sta_device_status().
+ *  - The library keeps one lazily grown device workspace per device (tile
+ *    lists and the work plan of sta_forward); calls that use it must not
+ *    overlap on different streams.  sta_shutdown() releases it.
+ */
+#ifndef STA_H_
+#define STA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum sta_status {
+  STA_OK = 0,
+  STA_ERR_INVALID_ARG = 1,    /* shape, window, text or pointer argument rejected  */
+  STA_ERR_UNSUPPORTED = 2,    /* legal STA but not built: d not in {64,128},
+                                 tile volume not a multiple of 128, not sm_100   */
+  STA_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed             */
+  STA_ERR_DEVICE_TIMEOUT = 4  /* a bounded device wait gave up (see above)       */
+} sta_status;
+
+/* Text block size (README Usage: "text tokens = 256 with padding"). */
+#define STA_TEXT_PAD 256
+
+/*
+ * sta_tile_reorder - raster -> tile token order (README Usage, "a tile is a
+ * cube"; tiles must be contiguous rows for the blocks of "Why is STA Fast?"
+ * to be dense).  Video row r = (t*H + h)*W + w moves to row
+ * tile_id*V + in_tile, tile_id = ((t/ct)*NH + h/ch)*NW + w/cw,
+ * in_tile = ((t%ct)*ch + h%ch)*cw + w%cw, V = ct*ch*cw.  Text rows are copied
+ * unchanged.  in/out: [B, heads, S, d] bf16 device, d in {64,128}
+ * (any d with d*2 % 16 == 0 is accepted).  Bit-exact copy.
+ */
+sta_status sta_tile_reorder(const void* in, void* out, int B, int heads, int d,
+                            int T, int H, int W, const int tile[3],
+                            int has_text, void* stream);
+
+/* sta_tile_unreorder - inverse of sta_tile_reorder (tile -> raster order). */
+sta_status sta_tile_unreorder(const void* in, void* out, int B, int heads,
+                              int d, int T, int H, int W, const int tile[3],
+                              int has_text, void* stream);
+
+/*
+ * sta_build_kv_tile_lists - per-query-tile KV tile lists (README Usage,
+ * "window_size in tiles": one (wt,wh,ww) per head).
+ *   counts: device int32 [heads][NQ], NQ = NV + (has_text ? 1 : 0),
+ *           NV = (T/ct)*(H/ch)*(W/cw)
+ *   ids:    device int32 [heads][NQ][max_k]
+ * Row r < NV: ascending ids of the key tiles inside query tile r's window,
+ * then the text sentinel NV when has_text && text_len > 0.  Row NV (text
+ * queries, only when has_text): 0..NV-1, then NV when text_len > 0.  Unused
+ * slots are -1.  window: HOST int32 [heads][3], each entry >= 1 (a window
+ * longer than the grid covers the axis).  max_k must be >= the longest row,
+ * else STA_ERR_INVALID_ARG.  Integer, bit-exact.
+ */
+sta_status sta_build_kv_tile_lists(int* counts, int* ids, int max_k, int heads,
+                                   int T, int H, int W, const int tile[3],
+                                   const int* window, int text_len,
+                                   int has_text, void* stream);
+
+/*
+ * sta_forward - fused STA attention, tile-ordered q,k,v -> out.
+ *   q, k, v: [B, heads, S, d] bf16 device, TILE order (sta_tile_reorder)
+ *   out:     [B, heads, S, d] bf16 device, tile order
+ *   d in {64, 128}; tile volume ct*ch*cw a multiple of 128;
+ *   window: HOST int32 [heads][3]; 0 <= text_len <= 256 (ignored when
+ *   has_text == 0).  Scale 1/sqrt(d).  bf16 inputs, fp32 accumulation and
+ *   softmax, probabilities rounded to bf16 for the P.V product, output
+ *   rounded to nearest even.  Runs on sm_100 only (tcgen05 / TMEM / TMA).
+ */
+sta_status sta_forward(const void* q, const void* k, const void* v, void* out,
+                       int B, int heads, int d, int T, int H, int W,
+                       const int tile[3], const int* window, int text_len,
+                       int has_text, void* stream);
+
+/* sta_forward_lse - sta_forward that also writes the natural-log
+ * log-sum-exp of every query row to `lse` (device fp32 [B, heads, S]). */
+sta_status sta_forward_lse(const void* q, const void* k, const void* v,
+                           void* out, float* lse, int B, int heads, int d,
+                           int T, int H, int W, const int tile[3],
+                           const int* window, int text_len, int has_text,
+                           void* stream);
+
+/*
+ * sta_swa_forward - token-level sliding-window attention with grouped-query
+ * heads, the mixed-block baseline of README "Why is STA Fast?"; the 1-D
+ * causal window over the previous `window` positions (self included) with
+ * GQA follows the sliding-window search-result page (Mistral 7B, 4096).
+ *   q:    [B, hq, S, d] bf16 device;  k, v: [B, hkv, S, d];  out like q
+ *   hq % hkv == 0, query head h reads KV head h / (hq/hkv);
+ *   S % 128 == 0, d in {64,128}, window >= 1, causal must be 1.
+ * Blocks of 128 keys fully outside the band are skipped, fully inside are
+ * dense, and only the blocks cut by the band edges are masked per element.
+ */
+sta_status sta_swa_forward(const void* q, const void* k, const void* v,
+                           void* out, int B, int hq, int hkv, int d, int S,
+                           int window, int causal, void* stream);
+
+/* Synchronises `stream`, returns STA_ERR_DEVICE_TIMEOUT if any kernel of this
+ * library recorded a gave-up wait since the last call (and clears it), else
+ * STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
+sta_status sta_device_status(void* stream);
+
+/* Static, never NULL. */
+const char* sta_status_string(sta_status s);
+
+/* Releases the per-device workspaces and cached plans. */
+void sta_shutdown(void);
+
+/* Effective work of sta_forward: allowed (query, key) pairs over all
+ * B*heads, counted on the host from the geometry (FLOPs = 4 * d * pairs). */
+int64_t sta_retained_pairs(int B, int heads, int T, int H, int W,
+                           const int tile[3], const int* window, int text_len,
+                           int has_text);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STA_H_ */
