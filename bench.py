@@ -1,0 +1,411 @@
+"""Benchmark of the STA forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one pass of the whole hot path on the video+text workload
+(B=1, 24 heads, d=128, video (30,48,80) in (6,8,8) tiles + 256 text tokens,
+text_length 200, window (3,3,3) tiles; inputs q, k, v bf16 N(0,1), seeded):
+  tile reorder of q, k, v -> KV tile lists + fused attention -> unreorder.
+The metric is effective TFLOP/s counting only retained (query, key) pairs,
+4 * d FLOP each.  Inputs (3 x 710 MB) are larger than L2, so no flush is
+needed between steps.
+
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch element
+of the same workload (independent problems, weak scaling, no data-path
+collective); the time is the max over ranks.
+
+--impl reference times the float64 CPU oracle on the host cores on a bounded
+sample of the same workload (it is the baseline, not the target).
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "STA forward ms and effective TFLOP/s (retained tiles) as % of B200 BF16 peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+ATTN_SOURCES = ("block_sparse_local_b200/csrc/attn_fwd.cuh",
+                "block_sparse_local_b200/csrc/device_ptx.cuh")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in ATTN_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def attn_traffic(units_per_launch):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, or None when the kernel source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "attn_fwd_video_text_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_hash") != source_hash():
+        return None
+    # captured on a smaller case; traffic scales with the key blocks processed
+    return d["dram_bytes_per_unit"] * units_per_launch
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        self.proc.wait()
+        sms, maxs, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sms.append(float(parts[1]))
+                    maxs.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        load = [s for s in sms if s > 600] or sms
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(maxs) if maxs else None,
+                "samples": len(sms), "reasons": sorted(reasons)}
+
+
+def cpu_oracle_sample(w, q_h, k_h, v_h, seconds):
+    """Time the float64 oracle (form B) on query tiles of one head until
+    ``seconds`` pass; returns (effective TFLOP/s, description, threads)."""
+    import numpy as np
+    from oracle import sta_oracle
+
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        threads = len(os.sched_getaffinity(0))
+    q64, k64, v64 = (x.double().numpy() for x in (q_h, k_h, v_h))
+    ct, ch, cw = w.tile
+    NT, NH, NW = w.T // ct, w.H // ch, w.W // cw
+    tiles_done, pairs, rows_done = 0, 0, 0
+    t0 = time.perf_counter()
+    for tq in range(NT * NH * NW):
+        qt, qh, qw = tq // (NH * NW), (tq // NW) % NH, tq % NW
+        tt = np.arange(qt * ct, (qt + 1) * ct)
+        hh = np.arange(qh * ch, (qh + 1) * ch)
+        ww = np.arange(qw * cw, (qw + 1) * cw)
+        rows = ((tt[:, None, None] * w.H + hh[None, :, None]) * w.W + ww[None, None, :]).ravel()
+        sta_oracle.sta_forward_rows(q64, k64, v64, w.T, w.H, w.W, w.tile, w.windows[0],
+                                    w.text_len, w.has_text, rows=rows)
+        keys = len(sta_oracle.allowed_keys(int(rows[0]), w.T, w.H, w.W, w.tile, w.windows[0],
+                                           w.text_len, w.has_text))
+        pairs += len(rows) * keys
+        rows_done += len(rows)
+        tiles_done += 1
+        if time.perf_counter() - t0 > seconds:
+            break
+    dt = time.perf_counter() - t0
+    tflops = 4.0 * w.d * pairs / dt / 1e12
+    desc = (f"float64 oracle (row-gather form) on {tiles_done} video query tiles "
+            f"({rows_done} rows) of head 0 of the same workload, {dt:.1f} s")
+    return tflops, desc, threads, dt
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as it stands, rank 0 only."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    from block_sparse_local_b200 import workloads
+
+    w = workloads.VIDEO_TEXT
+    g = torch.Generator().manual_seed(w.seed * 1000)
+    shape = (w.S, w.d)
+    q_h, k_h, v_h = (torch.randn(shape, generator=g).mul_(w.std).to(torch.bfloat16)
+                     for _ in range(3))
+    per_step = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, q_h, k_h, v_h, per_step / 4)
+    vals, total = [], 0.0
+    for _ in range(args.steps):
+        tf, desc, threads, dt = cpu_oracle_sample(w, q_h, k_h, v_h, per_step)
+        vals.append(tf)
+        total += dt
+    value = statistics.median(vals)
+    from oracle import sta_oracle
+    flops = 4.0 * w.d * sum(sta_oracle.retained_pairs(w.T, w.H, w.W, w.tile, tuple(win),
+                                                      w.text_len, w.has_text)
+                            for win in w.windows)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": flops / (value * 1e12) * 1e3 if value > 0 else None,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d,
+                   "video": [w.T, w.H, w.W], "tile": list(w.tile), "window": list(w.windows[0]),
+                   "text_len": w.text_len, "seq_len": w.S, "note": "ms_per_step extrapolated"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line))
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_local_b200 as sta
+    from block_sparse_local_b200 import workloads
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    w = workloads.VIDEO_TEXT
+    shape = (w.T, w.H, w.W)
+    # each rank draws its own batch element (independent problems)
+    gq = torch.Generator(device=dev)
+    qkv = []
+    for i in range(3):
+        gq.manual_seed(w.seed * 1000 + i + 17 * rank)
+        qkv.append(torch.randn((w.B, w.heads, w.S, w.d), generator=gq, device=dev,
+                               dtype=torch.float32).to(torch.bfloat16))
+    q, k, v = qkv
+    qt, kt, vt, ot, out = (torch.empty_like(q) for _ in range(5))
+    stream = torch.cuda.current_stream(dev)
+    pairs = sta.retained_pairs(w.B, w.windows, shape, w.tile, w.text_len, w.has_text)
+    flops = 4.0 * w.d * pairs
+
+    attn_ev = []
+
+    def step(record=False):
+        sta.tile_reorder(q, shape, w.tile, w.has_text, out=qt)
+        sta.tile_reorder(k, shape, w.tile, w.has_text, out=kt)
+        sta.tile_reorder(v, shape, w.tile, w.has_text, out=vt)
+        if record:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        sta.forward(qt, kt, vt, w.windows, w.text_len, w.has_text, shape, w.tile, out=ot)
+        if record:
+            e1.record(stream)
+            attn_ev.append((e0, e1))
+        sta.tile_unreorder(ot, shape, w.tile, w.has_text, out=out)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    sta.device_status(dev)
+    barrier()
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(record=True)
+    t1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    sta.device_status(dev)
+    ms = t0.elapsed_time(t1) / args.steps
+    attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    if world > 1:
+        tt = torch.tensor([ms, attn_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, attn_ms = float(tt[0]), float(tt[1])
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+        hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+
+        def e2e_step():
+            dq, dk, dv = (x.to(dev, non_blocking=True) for x in (hq, hk, hv))
+            o = sta.sliding_tile_attention(dq, dk, dv, w.windows, w.text_len, w.has_text,
+                                           shape, w.tile)
+            hout.copy_(o, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_e2e = max(3, min(args.steps, 10))
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        barrier()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt[0])
+        nbytes = q.numel() * q.element_size()
+        e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * nbytes,
+               "d2h_bytes_per_step": nbytes}
+
+    # ---- token-level sliding-window comparison (mixed blocks), same kernel family
+    swa = None
+    if rank == 0:
+        sw = workloads.SWA_GQA
+        sq, sk, sv = workloads.swa_inputs(sw, device=dev)
+        so = torch.empty_like(sq)
+        for _ in range(3):
+            sta.swa_forward(sq, sk, sv, sw.window, True, out=so)
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(10):
+            sta.swa_forward(sq, sk, sv, sw.window, True, out=so)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        swa_ms = a.elapsed_time(b) / 10
+        s_pairs = sw.hq * (sw.window * (sw.window + 1) // 2 + (sw.S - sw.window) * sw.window)
+        swa_flops = 4.0 * sw.d * s_pairs
+        # STA on the same geometry with 3 heads: about the same retained FLOPs
+        wins3 = w.windows[:3]
+        m_q, m_k, m_v = (x[:, :3].contiguous() for x in (qt, kt, vt))
+        m_o = torch.empty_like(m_q)
+        for _ in range(3):
+            sta.forward(m_q, m_k, m_v, wins3, w.text_len, w.has_text, shape, w.tile, out=m_o)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(10):
+            sta.forward(m_q, m_k, m_v, wins3, w.text_len, w.has_text, shape, w.tile, out=m_o)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        sta3_ms = a.elapsed_time(b) / 10
+        sta3_flops = 4.0 * w.d * sta.retained_pairs(1, wins3, shape, w.tile, w.text_len,
+                                                    w.has_text)
+        sta.device_status(dev)
+        swa = {"workload": sw.name, "ms": swa_ms,
+               "effective_tflops": swa_flops / (swa_ms * 1e-3) / 1e12,
+               "sta_matched": {"heads": 3, "ms": sta3_ms,
+                               "effective_tflops": sta3_flops / (sta3_ms * 1e-3) / 1e12}}
+        del sq, sk, sv, so, m_q, m_k, m_v, m_o
+
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    # per-launch key blocks x query blocks processed (units of the traffic file)
+    units = pairs / (128 * 128)
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": attn_traffic(units),
+                "kernel": "attn_fwd_kernel<128,kSta>", "peak_source": peak_src + " burst bf16",
+                "attn_ms": attn_ms}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, desc, threads, _ = cpu_oracle_sample(w, q[0, 0].cpu(), k[0, 0].cpu(), v[0, 0].cpu(),
+                                                 args.cpu_seconds)
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": threads, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "B_per_gpu": w.B, "heads": w.heads, "d": w.d,
+                       "video": [w.T, w.H, w.W], "tile": list(w.tile),
+                       "window": list(w.windows[0]), "text_len": w.text_len,
+                       "seq_len": w.S, "global_batch": w.B * world,
+                       "parallelism": f"independent problems x{world}",
+                       "l2": "inputs larger than L2 (3 x 710 MB), no flush",
+                       "step": "reorder q,k,v + tile lists + fused attention + unreorder"},
+            "pct_of_bf16_peak": 100.0 * value / peak,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
+            "gpu_launches": 6 * args.steps, "swa_comparison": swa,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
