@@ -20,16 +20,16 @@ from .build import LIB_PATH
 __all__ = [
     "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
-    "retained_pairs", "STATUS",
+    "retained_pairs", "STATUS", "forward_noalloc",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
-          3: "STA_ERR_CUDA", 4: "STA_ERR_DEVICE_TIMEOUT"}
+          3: "STA_ERR_CUDA", 4: "STA_ERR_DEVICE_TIMEOUT", 5: "STA_ERR_SCRATCH_LIMIT"}
 
 EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
             "sta_device_status", "sta_status_string", "sta_shutdown",
-            "sta_retained_pairs")
+            "sta_retained_pairs", "sta_forward_noalloc")
 
 
 class StaError(RuntimeError):
@@ -64,6 +64,7 @@ def lib():
            ctypes.POINTER(ctypes.c_int), _I, _I, _P]
     L.sta_forward.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_forward_lse.argtypes = [_P, _P, _P, _P, _P] + fwd
+    L.sta_forward_noalloc.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_status_string.argtypes = [_I]
@@ -167,6 +168,22 @@ def forward(q, k, v, window_size, text_length, has_text, video_shape,
     _check(lib().sta_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d, T, H, W,
                              _I3(*tile), wins, int(text_length), int(has_text),
                              _stream(q)), "sta_forward")
+    return out
+
+
+def forward_noalloc(q, k, v, window_size, text_length, has_text, video_shape,
+                    tile=(6, 8, 8), out=None):
+    """Like forward(), through sta_forward_noalloc: the library allocates no
+    device memory (its scratch is a fixed 4 MiB array); for callers whose
+    memory pool owns the device or that cannot take cudaMalloc's implicit
+    synchronisation.  Calls that overlap on the GPU race on the shared array."""
+    _check_qkv(q, k, v)
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib().sta_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d, T, H, W,
+                                     _I3(*tile), _windows(window_size, nh), int(text_length),
+                                     int(has_text), _stream(q)), "sta_forward_noalloc")
     return out
 
 

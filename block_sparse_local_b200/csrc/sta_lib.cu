@@ -477,6 +477,112 @@ std::vector<WorkItem> plan_swa(int B, int hq, int hkv, int S, int window) {
   return items;
 }
 
+// ------------------------------------------------------------------ no-alloc
+// Fixed scratch for sta_forward_noalloc: tile lists and the work plan live in
+// this file-scope array instead of the lazily grown workspace.  Host code must
+// not pass `g_noalloc_scratch` itself to a kernel (on the host it names a
+// stand-in, not device memory): each device's address is looked up once with
+// cudaGetSymbolAddress while that device is current.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[STA_NOALLOC_SCRATCH_BYTES];
+
+struct NoAllocState {
+  bool ready = false;
+  unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch
+  std::string plan_key;               // host-side plan cache (host memory only)
+  std::vector<WorkItem> items;
+};
+NoAllocState g_noalloc[64];
+
+sta_status forward_noalloc_impl(const void* q, const void* k, const void* v, void* out,
+                                int B, int heads, int d, int T, int H, int W,
+                                const int tile[3], const int* window, int text_len,
+                                int has_text, void* stream) {
+  if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1) return STA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return STA_ERR_INVALID_ARG;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, text_len);
+  if (s != STA_OK) return s;
+  s = check_windows(window, heads);
+  if (s != STA_OK) return s;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  if (g.V % sta::kBM != 0) return STA_ERR_UNSUPPORTED;
+  const int64_t total_rows = int64_t(B) * heads * g.S;
+  if (total_rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  Classes cls = make_classes(window, heads);
+  if (cls.nclass > kMaxClasses) return STA_ERR_UNSUPPORTED;
+  const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
+  int max_k = 1;
+  for (int c = 0; c < cls.nclass; ++c)
+    max_k = std::max(max_k, class_video_tiles(g, &cls.win[3 * c]) + sentinel);
+  if (g.has_text) max_k = std::max(max_k, g.NV + sentinel);
+  const int NQ = g.NV + (g.has_text ? 1 : 0);
+  const size_t counts_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
+  const size_t ids_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
+  // Size check from the geometry alone, before any plan is built.
+  const int bpt = g.V / sta::kBM;
+  const size_t max_items = size_t(B) * heads * (size_t(g.NV) * ((bpt + 1) / 2) + 1);
+  if (counts_bytes + ids_bytes + sizeof(WorkItem) * max_items > STA_NOALLOC_SCRATCH_BYTES)
+    return STA_ERR_SCRATCH_LIMIT;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+
+  std::lock_guard<std::mutex> lock(g_mu);
+  NoAllocState& na = g_noalloc[dev];
+  if (!na.ready) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr)
+      return STA_ERR_CUDA;
+    na.scratch = static_cast<unsigned char*>(ptr);
+    na.ready = true;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const std::string key = sta_key(dev, B, heads, d, g, window);
+  if (na.plan_key != key) {
+    na.items = plan_sta(g, cls, B, heads, max_k, nullptr);
+    na.plan_key = key;
+  }
+  const size_t items_bytes = sizeof(WorkItem) * na.items.size();
+  if (counts_bytes + ids_bytes + items_bytes > STA_NOALLOC_SCRATCH_BYTES)
+    return STA_ERR_SCRATCH_LIMIT;
+  int* d_counts = reinterpret_cast<int*>(na.scratch);
+  int* d_ids = reinterpret_cast<int*>(na.scratch + counts_bytes);
+  WorkItem* d_items = reinterpret_cast<WorkItem*>(na.scratch + counts_bytes + ids_bytes);
+
+  CUtensorMap mq, mk, mv;
+  s = make_row_map(&mq, q, total_rows, d);
+  if (s == STA_OK) s = make_row_map(&mk, k, total_rows, d);
+  if (s == STA_OK) s = make_row_map(&mv, v, total_rows, d);
+  if (s != STA_OK) return s;
+  // The array keeps the previous call's contents: the plan is rewritten on
+  // every call, and the list kernel rewrites every count and id it reads.
+  STA_CUDA_TRY(cudaMemcpyAsync(d_items, na.items.data(), items_bytes, cudaMemcpyHostToDevice, st));
+  launch_lists(d_counts, d_ids, cls, g, max_k, st);
+  STA_CUDA_TRY(cudaGetLastError());
+
+  FwdParams prm;
+  prm.items = d_items;
+  prm.counts = d_counts;
+  prm.ids = d_ids;
+  prm.max_k = max_k;
+  prm.tile_blocks = bpt;
+  prm.V = g.V;
+  prm.L_v = g.Lv;
+  prm.text_len = g.text_len;
+  prm.text_blocks = (g.text_len + sta::kBN - 1) / sta::kBN;
+  prm.text_sentinel = sentinel;
+  prm.window = 0;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = nullptr;
+  const int num_items = static_cast<int>(na.items.size());
+  if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+  return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -489,6 +595,8 @@ const char* sta_status_string(sta_status s) {
     case STA_ERR_UNSUPPORTED: return "STA_ERR_UNSUPPORTED: shape or device not supported";
     case STA_ERR_CUDA: return "STA_ERR_CUDA: a CUDA call failed";
     case STA_ERR_DEVICE_TIMEOUT: return "STA_ERR_DEVICE_TIMEOUT: a device wait gave up";
+    case STA_ERR_SCRATCH_LIMIT:
+      return "STA_ERR_SCRATCH_LIMIT: problem needs more than the fixed no-alloc scratch";
   }
   return "STA_ERR_UNKNOWN";
 }
@@ -539,6 +647,13 @@ sta_status sta_forward(const void* q, const void* k, const void* v, void* out, i
                        const int* window, int text_len, int has_text, void* stream) {
   return forward_impl(q, k, v, out, nullptr, B, heads, d, T, H, W, tile, window, text_len,
                       has_text, stream);
+}
+
+sta_status sta_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B,
+                               int heads, int d, int T, int H, int W, const int tile[3],
+                               const int* window, int text_len, int has_text, void* stream) {
+  return forward_noalloc_impl(q, k, v, out, B, heads, d, T, H, W, tile, window, text_len,
+                              has_text, stream);
 }
 
 sta_status sta_forward_lse(const void* q, const void* k, const void* v, void* out, float* lse,

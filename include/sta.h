@@ -44,7 +44,9 @@ typedef enum sta_status {
   STA_ERR_UNSUPPORTED = 2,    /* legal STA but not built: d not in {64,128},
                                  tile volume not a multiple of 128, not sm_100   */
   STA_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed             */
-  STA_ERR_DEVICE_TIMEOUT = 4  /* a bounded device wait gave up (see above)       */
+  STA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device wait gave up (see above)       */
+  STA_ERR_SCRATCH_LIMIT = 5   /* sta_forward_noalloc: the problem needs more than
+                                 STA_NOALLOC_SCRATCH_BYTES of scratch            */
 } sta_status;
 
 /* Text block size (README Usage: "text tokens = 256 with padding"). */
@@ -140,6 +142,39 @@ void sta_shutdown(void);
 int64_t sta_retained_pairs(int B, int heads, int T, int H, int W,
                            const int tile[3], const int* window, int text_len,
                            int has_text);
+
+/* Size of the fixed scratch array used by sta_forward_noalloc (4 MiB). */
+#define STA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * sta_forward_noalloc - sta_forward that never allocates memory.  No passage
+ * of the STA pages corresponds to it: it exists for callers that cannot let
+ * a library call cudaMalloc, e.g. a serving runtime whose memory pool owns
+ * the whole device (a stray cudaMalloc can fail or fragment it) or a
+ * latency-bound loop that cannot take the implicit device synchronisation of
+ * cudaMalloc / cudaFree.
+ *
+ * Same arguments, layout, numerics and errors as sta_forward.  The scratch
+ * that sta_forward keeps in its lazily grown workspace (KV tile lists and the
+ * work plan) lives instead in one file-scope device array of
+ * STA_NOALLOC_SCRATCH_BYTES, which every GPU that loads libsta.so holds until
+ * the process exits.  A problem whose tile lists and plan do not fit returns
+ * STA_ERR_SCRATCH_LIMIT before anything is enqueued (the video+text workload
+ * of 115,456 tokens x 24 heads needs about 0.55 MiB).
+ *
+ * The first call on a device looks up that device's address of the array
+ * (cudaGetSymbolAddress, with the device current), so make the first call on
+ * each device outside any stream capture.  All calls share the one array and
+ * it keeps the last call's contents; every call rewrites what it reads, so
+ * nothing needs clearing, but calls that overlap on the GPU (different
+ * streams, or several host threads) race on it: order them on one stream.
+ * It calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+sta_status sta_forward_noalloc(const void* q, const void* k, const void* v,
+                               void* out, int B, int heads, int d, int T,
+                               int H, int W, const int tile[3],
+                               const int* window, int text_len, int has_text,
+                               void* stream);
 
 #ifdef __cplusplus
 }
