@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-swa", action="store_true", help="skip the SWA comparison")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run the workload with fewer heads (profiling captures only)")
     return ap.parse_args()
 
 
@@ -231,6 +234,10 @@ def run_ours(args):
         dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     w = workloads.VIDEO_TEXT
+    if args.heads is not None:
+        import dataclasses
+        w = dataclasses.replace(w, name=f"{w.name}_heads{args.heads}", heads=args.heads,
+                                windows=w.windows[:1] * args.heads)
     shape = (w.T, w.H, w.W)
     # each rank draws its own batch element (independent problems)
     gq = torch.Generator(device=dev)
@@ -322,7 +329,7 @@ def run_ours(args):
 
     # ---- token-level sliding-window comparison (mixed blocks), same kernel family
     swa = None
-    if rank == 0:
+    if rank == 0 and not args.no_swa:
         sw = workloads.SWA_GQA
         sq, sk, sv = workloads.swa_inputs(sw, device=dev)
         so = torch.empty_like(sq)
