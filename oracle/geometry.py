@@ -11,7 +11,10 @@ README "Sliding Tile Atteniton Kernel", section Usage:
 
 Readings taken where the page is silent (each is listed in the design doc):
   * the window is centred on the query tile, start = c - floor(w/2), and
-    shifted inward at the grid border so that it always spans w tiles;
+    shifted inward at the grid border so that it always spans w tiles
+    (pinned for odd windows by the hand-derived fixtures; for an even window
+    shorter than the grid the choice of the extra tile on the low side is
+    parity unpinned: no page example fixes it);
   * a window longer than the grid axis is clipped to the whole axis;
   * with has_text=False there are no text rows at all.
 """
