@@ -20,7 +20,7 @@ from .build import LIB_PATH
 __all__ = [
     "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
-    "retained_pairs", "STATUS", "forward_noalloc",
+    "retained_pairs", "STATUS", "forward_noalloc", "forward_raster",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -29,7 +29,7 @@ STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
 EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
             "sta_device_status", "sta_status_string", "sta_shutdown",
-            "sta_retained_pairs", "sta_forward_noalloc")
+            "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster")
 
 
 class StaError(RuntimeError):
@@ -65,6 +65,7 @@ def lib():
     L.sta_forward.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_forward_lse.argtypes = [_P, _P, _P, _P, _P] + fwd
     L.sta_forward_noalloc.argtypes = [_P, _P, _P, _P] + fwd
+    L.sta_forward_raster.argtypes = [_P, _P, _P, _P, _P] + fwd
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_status_string.argtypes = [_I]
@@ -187,9 +188,38 @@ def forward_noalloc(q, k, v, window_size, text_length, has_text, video_shape,
     return out
 
 
+def forward_raster(q, k, v, window_size, text_length, has_text, video_shape,
+                   tile=(6, 8, 8), out=None, return_lse=False):
+    """STA attention on RASTER-ordered q, k, v with the permutation fused into
+    the kernel (sta_forward_raster).  Raises StaError(STA_ERR_UNSUPPORTED) when
+    a 128-row block of a tile is not a box of the grid."""
+    _check_qkv(q, k, v)
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, nh, S), dtype=torch.float32, device=q.device) if return_lse else None
+    _check(lib().sta_forward_raster(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                    None if lse is None else _ptr(lse), B, nh, d, T, H, W,
+                                    _I3(*tile), _windows(window_size, nh), int(text_length),
+                                    int(has_text), _stream(q)), "sta_forward_raster")
+    return (out, lse) if return_lse else out
+
+
 def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
-                           video_shape=(30, 48, 80), tile=(6, 8, 8)):
-    """README-style call on RASTER-ordered q, k, v: reorder, attend, unreorder."""
+                           video_shape=(30, 48, 80), tile=(6, 8, 8), fused=True):
+    """README-style call on RASTER-ordered q, k, v.
+
+    fused=True: one attention kernel reads and writes raster order directly
+    (sta_forward_raster); tile shapes whose blocks are not boxes of the grid
+    go through the explicit reorder -> attend -> unreorder kernels instead.
+    """
+    if fused:
+        try:
+            return forward_raster(q, k, v, window_size, text_length, has_text, video_shape,
+                                  tile)
+        except StaError as e:
+            if e.code != 2:
+                raise
     qt = tile_reorder(q, video_shape, tile, has_text)
     kt = tile_reorder(k, video_shape, tile, has_text)
     vt = tile_reorder(v, video_shape, tile, has_text)

@@ -34,13 +34,21 @@
 // reads P_i; tcgen05 MMAs of one thread execute in issue order.
 #pragma once
 
+#include <type_traits>
+
 #include "device_ptx.cuh"
 
 namespace sta {
 
 constexpr int kBM = 128;        // query rows per block (MMA M)
 constexpr int kBN = 128;        // keys per block
-constexpr int kFwdThreads = 320;
+// Warps that share one query row's softmax (each takes 128 / kSplit score
+// columns of the row); the two slots' softmax use 8 * kSplit warps.
+#ifndef STA_SOFTMAX_SPLIT
+#define STA_SOFTMAX_SPLIT 2
+#endif
+constexpr int kSplit = STA_SOFTMAX_SPLIT;
+constexpr int kFwdThreads = 64 + 256 * kSplit;
 constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpSoftmax0 = 2;
@@ -52,6 +60,17 @@ struct WorkItem {
   int q1;       // same for block 1, or -1
   int kv_base;  // first row of the key/value slice
   int list;     // kSta: tile-list row; kSwa: query block index
+};
+
+// Geometry of raster-ordered q, k, v, out (sta_forward_raster): the kernel
+// reads each 128-row block of a tile as a box of the (T, H, W) grid and
+// writes each output row to its raster position, so no separate permutation
+// pass is needed.
+struct RasterGeom {
+  int S;            // rows per (batch, head) slice
+  int ct, ch, cw;   // tile
+  int H, W;         // video grid (T is implied)
+  int NH, NW;       // tile grid
 };
 
 struct FwdParams {
@@ -69,6 +88,7 @@ struct FwdParams {
   float scale_log2;   // log2(e) / sqrt(d)
   __nv_bfloat16* out;
   float* lse;
+  RasterGeom rg;      // used when the kernel runs on raster-ordered tensors
 };
 
 template <int D>
@@ -82,7 +102,9 @@ struct FwdCfg {
   static constexpr int kKOff = kQOff + 2 * kBlockBytes;
   static constexpr int kVOff = kKOff + kKStages * kBlockBytes;
   static constexpr int kBarOff = kVOff + kVStages * kBlockBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;  // + barriers, align
+  static constexpr int kRedOff = kBarOff + 512;   // row-max / row-sum exchange
+  static constexpr int kRedBytes = 2 * 2 * 2 * kBM * 4;
+  static constexpr int kSmemBytes = kRedOff + kRedBytes + 1024;  // + 1024-byte align
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
 };
@@ -167,11 +189,75 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-template <int D, Mode M>
+// Pairs of score columns (of the 16 pairs of each 32-column group) whose
+// exp2 is evaluated by exp2_poly on the FMA pipe instead of MUFU, spread
+// evenly; unmasked blocks only.
+#ifndef STA_EXP2_POLY_PAIRS
+#define STA_EXP2_POLY_PAIRS 0
+#endif
+__device__ __forceinline__ constexpr bool kPolyPair(int e) {
+  return (e * STA_EXP2_POLY_PAIRS) % 16 >= 16 - STA_EXP2_POLY_PAIRS;
+}
+
+// Loads one 128-row block whose first row in the tile-ordered view is `row`
+// (kPanels loads of 128 rows x 128 bytes).  Tile-ordered tensors and the text
+// block: rows of the 2-D [B*heads*S, d] view.  Video blocks of raster-ordered
+// tensors (R): the block is a box of its tile in the (d, W, H, T, slice) view;
+// the box lands in shared memory in the tile's own (t, h, w) order.
+template <int D, bool R>
+__device__ __forceinline__ void load_block(uint8_t* dst, const CUtensorMap* m2,
+                                           const CUtensorMap* m5, uint64_t* bar, int row,
+                                           const FwdParams& p, uint64_t pol) {
+  constexpr int kPanels = D / 64;
+  if constexpr (R) {
+    const RasterGeom& g = p.rg;
+    const int slice = row / g.S;
+    const int off = row - slice * g.S;
+    if (off < p.L_v) {
+      const int tile = off / p.V;
+      const int ins = off - tile * p.V;
+      const int it = ins / (g.ch * g.cw);
+      const int ih = (ins / g.cw) % g.ch;
+      const int tw = tile % g.NW;
+      const int th = (tile / g.NW) % g.NH;
+      const int tt = tile / (g.NW * g.NH);
+#pragma unroll
+      for (int pn = 0; pn < kPanels; ++pn)
+        tma_load_5d(dst + pn * 128 * 128, m5, bar, pn * 64, tw * g.cw, th * g.ch + ih,
+                    tt * g.ct + it, slice, pol);
+      return;
+    }
+  }
+#pragma unroll
+  for (int pn = 0; pn < kPanels; ++pn)
+    tma_load_2d_hint(dst + pn * 128 * 128, m2, bar, pn * 64, row, pol);
+}
+
+// Raster row of tile-ordered row `row` (identity for text rows).
+__device__ __forceinline__ int raster_row(const FwdParams& p, int row) {
+  const RasterGeom& g = p.rg;
+  const int slice = row / g.S;
+  const int off = row - slice * g.S;
+  if (off >= p.L_v) return row;
+  const int tile = off / p.V;
+  const int ins = off - tile * p.V;
+  const int it = ins / (g.ch * g.cw);
+  const int ih = (ins / g.cw) % g.ch;
+  const int iw = ins % g.cw;
+  const int tw = tile % g.NW;
+  const int th = (tile / g.NW) % g.NH;
+  const int tt = tile / (g.NW * g.NH);
+  return slice * g.S + ((tt * g.ct + it) * g.H + th * g.ch + ih) * g.W + tw * g.cw + iw;
+}
+
+template <int D, Mode M, bool R>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_q5,
+                    const __grid_constant__ CUtensorMap tmap_k5,
+                    const __grid_constant__ CUtensorMap tmap_v5,
                     const FwdParams p) {
   using C = FwdCfg<D>;
   constexpr int KST = C::kKStages;
@@ -189,7 +275,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_full = s_full + 2;      // [2]
   uint64_t* o_full = p_full + 2;      // [2]
   uint64_t* mma_done = o_full + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  uint64_t* xbar = mma_done + 1;      // [2 slots][4 lane quarters] exchange
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xbar + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -205,10 +292,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     for (int i = 0; i < VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 4);
+      mbar_init(&p_full[i], 4 * kSplit);
       mbar_init(&o_full[i], 1);
     }
     mbar_init(mma_done, 1);
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 32 * kSplit);
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
     fence_mbar_init();
   }
@@ -216,6 +304,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
+    if constexpr (R) {
+      tma_prefetch_desc(&tmap_q5);
+      tma_prefetch_desc(&tmap_k5);
+      tma_prefetch_desc(&tmap_v5);
+    }
   }
   if (warp == kWarpMma) tmem_alloc(tmem_holder, C::kTmemCols);
   tc_fence_before();
@@ -232,13 +325,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------ producer
     if (lane == 0 && !skip) {
       const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
       mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
       for (int s = 0; s < (two ? 2 : 1); ++s) {
         const int qrow = s ? item.q1 : item.q0;
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d(smem + C::kQOff + s * C::kBlockBytes + pn * C::kPanelBytes,
-                      &tmap_q, q_full, pn * 64, qrow);
+        load_block<D, R>(smem + C::kQOff + s * C::kBlockBytes, &tmap_q, &tmap_q5, q_full, qrow,
+                         p, pol_q);
       }
       int issued = 0;
       for (int j = 0; j < n; ++j) {
@@ -246,20 +338,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, abort_flag)) break;
         const int row = seq_row<M>(p, seq, j);
         mbar_arrive_expect_tx(&k_full[ks], C::kBlockBytes);
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d_hint(smem + C::kKOff + ks * C::kBlockBytes + pn * C::kPanelBytes,
-                           &tmap_k, &k_full[ks], pn * 64, row, pol_kv);
+        load_block<D, R>(smem + C::kKOff + ks * C::kBlockBytes, &tmap_k, &tmap_k5, &k_full[ks],
+                         row, p, pol_kv);
         const int vs = j % VST;
         if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, abort_flag)) {
           issued = j * 2 + 1;
           break;
         }
         mbar_arrive_expect_tx(&v_full[vs], C::kBlockBytes);
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn)
-          tma_load_2d_hint(smem + C::kVOff + vs * C::kBlockBytes + pn * C::kPanelBytes,
-                           &tmap_v, &v_full[vs], pn * 64, row, pol_kv);
+        load_block<D, R>(smem + C::kVOff + vs * C::kBlockBytes, &tmap_v, &tmap_v5, &v_full[vs],
+                         row, p, pol_kv);
         issued = j * 2 + 2;
       }
       // Leave no copy in flight: wait for the last load of every stage.
@@ -347,44 +435,67 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int slot = (warp - kWarpSoftmax0) >> 2;
+    // kSplit warps share each query row: warp k of the softmax warps serves
+    // slot k / (4 kSplit), column half (k / 4) % kSplit, TMEM lane quarter
+    // warp % 4.  With kSplit = 2 the halves exchange their partial row max
+    // every block (and their partial sums once, at the end) through shared
+    // memory behind an mbarrier.
+    constexpr int kCols = kBN / kSplit;       // score columns per thread
+    constexpr int kOCols = D / kSplit;        // output columns per thread
+    const int ks = warp - kWarpSoftmax0;
+    const int slot = ks / (4 * kSplit);
+    const int half = (ks / 4) % kSplit;
     const int sub = warp & 3;                 // TMEM lane quarter of this warp
     const int r = sub * 32 + lane;            // query row inside the block
+    float* red = reinterpret_cast<float*>(smem + C::kRedOff);   // [2][2][2][128]
+    uint64_t* xb = &xbar[slot * 4 + sub];
+    (void)red;
+    (void)xb;
     if (!skip && (slot == 0 || two)) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u);
-      const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0);
+      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u) + half * kCols;
+      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u) + half * (kCols / 2);
+      const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0) + half * kOCols;
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY;   // running max, log2 units of the scaled scores
-      float l_run = 0.f;
+      float l_run = 0.f;         // this thread's part of the row sum
       bool done = true;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
-        uint32_t sr[128];
-        STA_TMEM_LD32(t_s + 0, (sr + 0));
-        STA_TMEM_LD32(t_s + 32, (sr + 32));
-        STA_TMEM_LD32(t_s + 64, (sr + 64));
-        STA_TMEM_LD32(t_s + 96, (sr + 96));
+        uint32_t sr[kCols];
+#pragma unroll
+        for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_LD32(t_s + cc * 32, (sr + cc * 32));
         tmem_wait_ld();
-        float s[128];
+        float s[kCols];
 #pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+        for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
         int lo, hi;
-        if (seq_mask<M>(p, seq, j, r, lo, hi)) {
+        const bool masked = seq_mask<M>(p, seq, j, r, lo, hi);
+        if (masked) {
+          lo -= half * kCols;
+          hi -= half * kCols;
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
+          for (int c = 0; c < kCols; ++c)
             if (c < lo || c >= hi) s[c] = -INFINITY;
         }
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
+        for (int c = 4; c < kCols; c += 4) {
           mx0 = fmaxf(mx0, s[c]);
           mx1 = fmaxf(mx1, s[c + 1]);
           mx2 = fmaxf(mx2, s[c + 2]);
           mx3 = fmaxf(mx3, s[c + 3]);
         }
-        const float m_cand = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        if constexpr (kSplit == 2) {
+          float* rb = red + ((j & 1) * 2 + slot) * 2 * kBM;
+          rb[half * kBM + r] = mx;
+          mbar_arrive(xb);
+          if (!mbar_wait_warp(xb, j & 1, abort_flag)) { done = false; break; }
+          mx = fmaxf(mx, rb[(half ^ 1) * kBM + r]);
+        }
+        const float m_cand = mx * sl2;
         const bool resc = m_cand > m_run + 8.0f;
         float alpha = 1.f;
         if (resc) {
@@ -394,23 +505,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
         float ls0 = 0.f, ls1 = 0.f;
+        // exp2 of the scaled, shifted scores -> bf16 P in TMEM; on unmasked
+        // blocks a share of the pairs goes to the FMA-pipe polynomial.
+        auto exp_block = [&](auto use_poly) {
+          constexpr bool kPoly = decltype(use_poly)::value;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t pk[16];
+          for (int cc = 0; cc < kCols / 32; ++cc) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
-            const float p1 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
-            ls0 += p0;
-            ls1 += p1;
-            pk[e] = pack_bf16x2(p0, p1);
+            for (int e = 0; e < 16; ++e) {
+              const float x0 = fmaf(s[cc * 32 + 2 * e], sl2, neg_m);
+              const float x1 = fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m);
+              const bool poly = kPoly && kPolyPair(e);
+              const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
+              const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
+              ls0 += p0;
+              ls1 += p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            STA_TMEM_ST16(t_p + cc * 16, pk);
           }
-          STA_TMEM_ST16(t_s + cc * 16, pk);
+        };
+        if (masked) {
+          exp_block(std::false_type{});
+        } else {
+          exp_block(std::true_type{});
         }
         l_run += ls0 + ls1;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
+          for (int cc = 0; cc < kOCols / 32; ++cc) {
             uint32_t o[32];
             STA_TMEM_LD32(t_o + cc * 32, o);
             tmem_wait_ld();
@@ -426,27 +550,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (done && mbar_wait_warp(&o_full[slot], 0, abort_flag)) {
         tc_fence_after();
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        const int qrow = (slot ? item.q1 : item.q0) + r;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(qrow) * D);
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          STA_TMEM_LD32(t_o + cc * 32, o);
-          tmem_wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
-                                __uint_as_float(o[2 * e + 1]) * inv);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
-                                          pk[4 * v4 + 3]);
+        bool ok = true;
+        if constexpr (kSplit == 2) {
+          float* rb = red + ((n & 1) * 2 + slot) * 2 * kBM;
+          rb[half * kBM + r] = l_run;
+          mbar_arrive(xb);
+          ok = mbar_wait_warp(xb, n & 1, abort_flag);
+          if (ok) l_run += rb[(half ^ 1) * kBM + r];
         }
-        if (p.lse != nullptr) {
-          const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-          p.lse[qrow] = (m_use + __log2f(l_run)) * 0.69314718055994531f;
+        if (ok) {
+          const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+          int qrow = (slot ? item.q1 : item.q0) + r;
+          if constexpr (R) qrow = raster_row(p, qrow);
+          uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(qrow) * D +
+                                                half * kOCols);
+#pragma unroll
+          for (int cc = 0; cc < kOCols / 32; ++cc) {
+            uint32_t o[32];
+            STA_TMEM_LD32(t_o + cc * 32, o);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
+                                  __uint_as_float(o[2 * e + 1]) * inv);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                            pk[4 * v4 + 3]);
+          }
+          if (p.lse != nullptr && half == 0) {
+            const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+            p.lse[qrow] = (m_use + __log2f(l_run)) * 0.69314718055994531f;
+          }
         }
       }
     }

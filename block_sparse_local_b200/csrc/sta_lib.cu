@@ -97,6 +97,26 @@ sta_status make_row_map(CUtensorMap* map, const void* base, int64_t rows, int d)
   return r == CUDA_SUCCESS ? STA_OK : STA_ERR_CUDA;
 }
 
+// Raster-ordered [slices, T, H, W, d] bf16 viewed as (d, W, H, T, slice) with
+// slice stride S*d (the text rows sit between slices); box = one 128-row block
+// of a tile: {64, cw, bh, bt, 1} with cw*bh*bt = 128, 128-byte swizzle.
+sta_status make_raster_map(CUtensorMap* map, const void* base, int slices, int S, int T,
+                           int H, int W, int d, int cw, int bh, int bt) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return STA_ERR_CUDA;
+  const cuuint64_t e = 2;
+  cuuint64_t dims[5] = {cuuint64_t(d), cuuint64_t(W), cuuint64_t(H), cuuint64_t(T),
+                        cuuint64_t(slices)};
+  cuuint64_t strides[4] = {e * d, e * d * W, e * d * W * H, e * d * S};
+  cuuint32_t box[5] = {64, cuuint32_t(cw), cuuint32_t(bh), cuuint32_t(bt), 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims,
+                  strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? STA_OK : STA_ERR_CUDA;
+}
+
 // ------------------------------------------------------------------ geometry
 struct Geom {
   int T, H, W, ct, ch, cw;
@@ -302,26 +322,31 @@ std::string sta_key(int dev, int B, int heads, int d, const Geom& g, const int* 
   return k;
 }
 
-template <int D, Mode M>
+// mq5/mk5/mv5: 5-D maps of raster-ordered tensors (R), else unused copies.
+template <int D, Mode M, bool R = false>
 sta_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const FwdParams& prm, int num_items, cudaStream_t st) {
+                       const FwdParams& prm, int num_items, cudaStream_t st,
+                       const CUtensorMap* mq5 = nullptr, const CUtensorMap* mk5 = nullptr,
+                       const CUtensorMap* mv5 = nullptr) {
   constexpr int smem = sta::FwdCfg<D>::kSmemBytes;
   static bool attr_set[64] = {};
   int dev = 0;
   STA_CUDA_TRY(cudaGetDevice(&dev));
   if (!attr_set[dev]) {
-    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_fwd_kernel<D, M>,
+    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_fwd_kernel<D, M, R>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     attr_set[dev] = true;
   }
-  sta::attn_fwd_kernel<D, M><<<num_items, sta::kFwdThreads, smem, st>>>(mq, mk, mv, prm);
+  sta::attn_fwd_kernel<D, M, R><<<num_items, sta::kFwdThreads, smem, st>>>(
+      mq, mk, mv, mq5 ? *mq5 : mq, mk5 ? *mk5 : mk, mv5 ? *mv5 : mv, prm);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
 
 sta_status forward_impl(const void* q, const void* k, const void* v, void* out, float* lse,
                         int B, int heads, int d, int T, int H, int W, const int tile[3],
-                        const int* window, int text_len, int has_text, void* stream) {
+                        const int* window, int text_len, int has_text, void* stream,
+                        bool raster = false) {
   if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return STA_ERR_INVALID_ARG;
@@ -336,6 +361,16 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (g.V % sta::kBM != 0) return STA_ERR_UNSUPPORTED;
   const int64_t total_rows = int64_t(B) * heads * g.S;
   if (total_rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  // Raster order: a 128-row block of a tile must be a box {cw, bh, bt} of
+  // whole rows of the tile (cw | 128, and ch*cw | 128 or 128 | ch*cw).
+  int box_h = 0, box_t = 0;
+  if (raster) {
+    const int plane = g.ch * g.cw;
+    if (128 % g.cw != 0 || !(128 % plane == 0 || plane % 128 == 0)) return STA_ERR_UNSUPPORTED;
+    box_h = std::min(g.ch, 128 / g.cw);
+    box_t = 128 / (g.cw * box_h);
+    if (B * int64_t(heads) > (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  }
   int dev = 0;
   s = current_device(&dev);
   if (s != STA_OK) return s;
@@ -400,6 +435,21 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = lse;
+  prm.rg.S = g.S;
+  prm.rg.ct = g.ct; prm.rg.ch = g.ch; prm.rg.cw = g.cw;
+  prm.rg.H = g.H; prm.rg.W = g.W;
+  prm.rg.NH = g.NH; prm.rg.NW = g.NW;
+  if (raster) {
+    CUtensorMap q5, k5, v5;
+    const int slices = B * heads;
+    s = make_raster_map(&q5, q, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+    if (s == STA_OK) s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+    if (s == STA_OK) s = make_raster_map(&v5, v, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+    if (s != STA_OK) return s;
+    if (d == 128)
+      return launch_attn<128, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
+    return launch_attn<64, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
+  }
   if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
   return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
 }
@@ -647,6 +697,14 @@ sta_status sta_forward(const void* q, const void* k, const void* v, void* out, i
                        const int* window, int text_len, int has_text, void* stream) {
   return forward_impl(q, k, v, out, nullptr, B, heads, d, T, H, W, tile, window, text_len,
                       has_text, stream);
+}
+
+sta_status sta_forward_raster(const void* q, const void* k, const void* v, void* out,
+                              float* lse, int B, int heads, int d, int T, int H, int W,
+                              const int tile[3], const int* window, int text_len, int has_text,
+                              void* stream) {
+  return forward_impl(q, k, v, out, lse, B, heads, d, T, H, W, tile, window, text_len,
+                      has_text, stream, true);
 }
 
 sta_status sta_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B,

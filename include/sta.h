@@ -112,6 +112,23 @@ sta_status sta_forward_lse(const void* q, const void* k, const void* v,
                            void* stream);
 
 /*
+ * sta_forward_raster - sta_forward on RASTER-ordered tensors, the README's
+ * calling convention (Usage: q, k, v [batch, heads, T*H*W + 256, head_dim]
+ * in video order), with the raster <-> tile permutation fused into the
+ * attention kernel: each 128-row block of a tile is loaded as a box of the
+ * (T, H, W) grid by a 5-D TMA descriptor, and every output row is stored at
+ * its raster position.  Same arguments and numerics as sta_forward_lse;
+ * `lse` may be NULL (else device fp32 [B, heads, S], raster order).
+ * Requires cw | 128 and (ch*cw | 128 or 128 | ch*cw), else
+ * STA_ERR_UNSUPPORTED (use sta_tile_reorder + sta_forward + unreorder).
+ */
+sta_status sta_forward_raster(const void* q, const void* k, const void* v,
+                              void* out, float* lse, int B, int heads, int d,
+                              int T, int H, int W, const int tile[3],
+                              const int* window, int text_len, int has_text,
+                              void* stream);
+
+/*
  * sta_swa_forward - token-level sliding-window attention with grouped-query
  * heads, the mixed-block baseline of README "Why is STA Fast?"; the 1-D
  * causal window over the previous `window` positions (self included) with

@@ -117,3 +117,40 @@ def test_full_window_is_dense_attention():
     ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double())
     err = np.abs(got - ref.numpy())
     assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS
+
+
+RASTER_CASES = [
+    # (T,H,W), tile, windows, text_len, has_text, d, B
+    ((12, 16, 24), (6, 8, 8), [(2, 2, 2), (1, 1, 3)], 200, True, 128, 1),   # box 8x8x2
+    ((1, 64, 64), (1, 16, 16), [(1, 3, 3)], 0, False, 64, 2),               # box 16x8x1
+    ((4, 24, 32), (2, 8, 8), [(1, 3, 3), (2, 2, 4)], 37, True, 128, 1),      # 128-token tiles
+    ((8, 32, 16), (2, 16, 8), [(3, 1, 2)], 129, True, 64, 1),               # box 8x16x1
+]
+
+
+@pytest.mark.parametrize("case", RASTER_CASES, ids=lambda c: f"{c[0]}-{c[1]}-t{c[3]}-d{c[5]}")
+def test_fused_raster_forward_matches_oracle(case):
+    shape, tile, windows, text_len, has_text, d, B = case
+    w = workloads.small_sta_case(*shape, tile, windows, text_len, has_text, d=d, B=B, seed=17)
+    q, k, v = workloads.sta_inputs(w)
+    out, lse = sta.forward_raster(q.cuda(), k.cuda(), v.cuda(), w.windows, w.text_len,
+                                  w.has_text, shape, w.tile, return_lse=True)
+    sta.device_status()
+    res = _oracle(w, q, k, v)
+    _compare(out.float().cpu().numpy(), res)
+    for (b, h), (_, ref_lse) in res.items():
+        assert np.abs(lse[b, h].cpu().numpy() - ref_lse).max() < 1e-2
+
+
+def test_non_box_tiles_fall_back_to_reorder_kernels():
+    # 24 tokens along w do not divide a 128-row block: the fused raster path
+    # refuses it and sliding_tile_attention uses the explicit permutation.
+    w = workloads.small_sta_case(4, 4, 48, (4, 4, 24), [(1, 1, 2)], 0, False, d=64, seed=19)
+    q, k, v = workloads.sta_inputs(w)
+    with pytest.raises(sta.StaError) as err:
+        sta.forward_raster(q.cuda(), k.cuda(), v.cuda(), w.windows, 0, False, (4, 4, 48), w.tile)
+    assert err.value.code == 2
+    out = sta.sliding_tile_attention(q.cuda(), k.cuda(), v.cuda(), w.windows, 0, False,
+                                     (4, 4, 48), w.tile)
+    sta.device_status()
+    _compare(out.float().cpu().numpy(), _oracle(w, q, k, v))
