@@ -382,11 +382,27 @@ def run_ours(args):
         sta3_ms = a.elapsed_time(b) / 10
         sta3_flops = 4.0 * w.d * sta.retained_pairs(1, wins3, shape, w.tile, w.text_len,
                                                     w.has_text)
+        # token-level 3-D sliding window with the same (18,24,24)-token
+        # window on the same workload: identical retained pairs, mixed blocks
+        win_tok = tuple(wa * ta for wa, ta in zip(w.windows[0], w.tile))
+        for _ in range(2):
+            sta.swa3d_forward(q, k, v, win_tok, w.text_len, w.has_text, shape, w.tile, out=out)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(3):
+            sta.swa3d_forward(q, k, v, win_tok, w.text_len, w.has_text, shape, w.tile, out=out)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        s3_ms = a.elapsed_time(b) / 3
         sta.device_status(dev)
         swa = {"workload": sw.name, "ms": swa_ms,
                "effective_tflops": swa_flops / (swa_ms * 1e-3) / 1e12,
                "sta_matched": {"heads": 3, "ms": sta3_ms,
-                               "effective_tflops": sta3_flops / (sta3_ms * 1e-3) / 1e12}}
+                               "effective_tflops": sta3_flops / (sta3_ms * 1e-3) / 1e12},
+               "token_window_3d": {"workload": w.name, "window_tokens": list(win_tok),
+                                   "ms": s3_ms,
+                                   "effective_tflops": flops / (s3_ms * 1e-3) / 1e12,
+                                   "sta_speedup": s3_ms / ms}}
         del sq, sk, sv, so, m_q, m_k, m_v, m_o
 
     peaks, peak_src = load_peaks()

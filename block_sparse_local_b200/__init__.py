@@ -20,7 +20,7 @@ from .build import LIB_PATH
 __all__ = [
     "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
-    "retained_pairs", "STATUS", "forward_noalloc", "forward_raster",
+    "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -29,7 +29,8 @@ STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
 EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
             "sta_device_status", "sta_status_string", "sta_shutdown",
-            "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster")
+            "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
+            "sta_swa3d_forward")
 
 
 class StaError(RuntimeError):
@@ -66,6 +67,7 @@ def lib():
     L.sta_forward_lse.argtypes = [_P, _P, _P, _P, _P] + fwd
     L.sta_forward_noalloc.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_forward_raster.argtypes = [_P, _P, _P, _P, _P] + fwd
+    L.sta_swa3d_forward.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_status_string.argtypes = [_I]
@@ -225,6 +227,21 @@ def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
     vt = tile_reorder(v, video_shape, tile, has_text)
     ot = forward(qt, kt, vt, window_size, text_length, has_text, video_shape, tile)
     return tile_unreorder(ot, video_shape, tile, has_text)
+
+
+def swa3d_forward(q, k, v, window_tokens, text_length, has_text, video_shape,
+                  tile=(6, 8, 8), out=None):
+    """Token-level 3-D sliding-window attention on RASTER-ordered q, k, v:
+    each query sees a window of (Wt, Wh, Ww) tokens around it (the mixed-block
+    baseline of STA); tiles must have 8 x 8 tokens per t-slice."""
+    _check_qkv(q, k, v)
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib().sta_swa3d_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d, T, H, W,
+                                   _I3(*tile), _I3(*window_tokens), int(text_length),
+                                   int(has_text), _stream(q)), "sta_swa3d_forward")
+    return out
 
 
 def swa_forward(q, k, v, window, causal=True, out=None):

@@ -53,7 +53,7 @@ constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpSoftmax0 = 2;
 
-enum class Mode { kSta = 0, kSwa = 1 };
+enum class Mode { kSta = 0, kSwa = 1, kSwa3d = 2 };
 
 struct WorkItem {
   int q0;       // first row (in the [B*heads*S, d] view) of query block 0
@@ -68,6 +68,7 @@ struct WorkItem {
 // pass is needed.
 struct RasterGeom {
   int S;            // rows per (batch, head) slice
+  int T;            // video grid along t
   int ct, ch, cw;   // tile
   int H, W;         // video grid (T is implied)
   int NH, NW;       // tile grid
@@ -85,6 +86,7 @@ struct FwdParams {
   int text_blocks;    // key blocks of the text block holding valid keys
   int text_sentinel;  // lists end with the text block
   int window;         // kSwa: tokens
+  int win3[3];        // kSwa3d: (Wt, Wh, Ww) token window
   float scale_log2;   // log2(e) / sqrt(d)
   __nv_bfloat16* out;
   float* lse;
@@ -122,7 +124,7 @@ template <Mode M>
 __device__ __forceinline__ KvSeq make_seq(const FwdParams& p, const WorkItem& it) {
   KvSeq s;
   s.kv_base = it.kv_base;
-  if constexpr (M == Mode::kSta) {
+  if constexpr (M != Mode::kSwa) {
     const int cnt = p.counts[it.list];
     s.ids = p.ids + static_cast<size_t>(it.list) * p.max_k;
     s.nvid = (cnt - p.text_sentinel) * p.tile_blocks;
@@ -141,7 +143,7 @@ __device__ __forceinline__ KvSeq make_seq(const FwdParams& p, const WorkItem& it
 
 template <Mode M>
 __device__ __forceinline__ int seq_row(const FwdParams& p, const KvSeq& s, int j) {
-  if constexpr (M == Mode::kSta) {
+  if constexpr (M != Mode::kSwa) {
     if (j < s.nvid) {
       const int t = j / p.tile_blocks;
       return s.kv_base + s.ids[t] * p.V + (j - t * p.tile_blocks) * kBN;
@@ -157,7 +159,7 @@ __device__ __forceinline__ int seq_row(const FwdParams& p, const KvSeq& s, int j
 template <Mode M>
 __device__ __forceinline__ bool seq_mask(const FwdParams& p, const KvSeq& s, int j,
                                          int r, int& lo, int& hi) {
-  if constexpr (M == Mode::kSta) {
+  if constexpr (M != Mode::kSwa) {
     if (j < s.nvid) return false;
     const int col0 = (j - s.nvid) * kBN;
     if (col0 + kBN <= p.text_len) return false;
@@ -231,6 +233,27 @@ __device__ __forceinline__ void load_block(uint8_t* dst, const CUtensorMap* m2,
 #pragma unroll
   for (int pn = 0; pn < kPanels; ++pn)
     tma_load_2d_hint(dst + pn * 128 * 128, m2, bar, pn * 64, row, pol);
+}
+
+// kSwa3d, tiles with 8 x 8 tokens per t-slice: each 128-key block holds two
+// t-slices of 64 keys, one per softmax half.  Bit c of the result is set when
+// key c of this thread's half (in-tile order: c = 8*h + w) lies in the token
+// window [ws, ws + we) of the query along every axis.
+__device__ __forceinline__ uint64_t swa3d_half_mask(int key_t, int key_h0, int key_w0,
+                                                    const int ws[3], const int we[3]) {
+  if (key_t < ws[0] || key_t >= ws[0] + we[0]) return 0ull;
+  auto bits8 = [](int lo, int hi) -> uint32_t {
+    lo = lo < 0 ? 0 : (lo > 8 ? 8 : lo);
+    hi = hi < 0 ? 0 : (hi > 8 ? 8 : hi);
+    return hi > lo ? ((1u << hi) - 1u) & ~((1u << lo) - 1u) : 0u;
+  };
+  const uint32_t mh = bits8(ws[1] - key_h0, ws[1] + we[1] - key_h0);
+  const uint64_t mw = bits8(ws[2] - key_w0, ws[2] + we[2] - key_w0);
+  uint64_t m = 0;
+#pragma unroll
+  for (int ih = 0; ih < 8; ++ih)
+    if ((mh >> ih) & 1u) m |= mw << (8 * ih);
+  return m;
 }
 
 // Raster row of tile-ordered row `row` (identity for text rows).
@@ -460,6 +483,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float m_run = -INFINITY;   // running max, log2 units of the scaled scores
       float l_run = 0.f;         // this thread's part of the row sum
       bool done = true;
+      // kSwa3d: this query's token window (video rows only)
+      bool tok_row = false;
+      int tws[3] = {0, 0, 0}, twe[3] = {0, 0, 0};
+      if constexpr (M == Mode::kSwa3d) {
+        const int off = (slot ? item.q1 : item.q0) + r - item.kv_base;
+        if (off < p.L_v) {
+          const RasterGeom& g = p.rg;
+          const int tile = off / p.V;
+          const int ins = off - tile * p.V;
+          const int tw = tile % g.NW, th = (tile / g.NW) % g.NH, tt = tile / (g.NW * g.NH);
+          const int tok[3] = {tt * g.ct + ins / (g.ch * g.cw), th * g.ch + (ins / g.cw) % g.ch,
+                              tw * g.cw + ins % g.cw};
+          const int dim[3] = {g.T, g.H, g.W};
+#pragma unroll
+          for (int a = 0; a < 3; ++a) {
+            twe[a] = p.win3[a] < dim[a] ? p.win3[a] : dim[a];
+            int st = tok[a] - twe[a] / 2;
+            st = st < 0 ? 0 : (st > dim[a] - twe[a] ? dim[a] - twe[a] : st);
+            tws[a] = st;
+          }
+          tok_row = true;
+        }
+      }
+      (void)tok_row;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
@@ -471,13 +518,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
         int lo, hi;
-        const bool masked = seq_mask<M>(p, seq, j, r, lo, hi);
+        bool masked = seq_mask<M>(p, seq, j, r, lo, hi);
         if (masked) {
           lo -= half * kCols;
           hi -= half * kCols;
 #pragma unroll
           for (int c = 0; c < kCols; ++c)
             if (c < lo || c >= hi) s[c] = -INFINITY;
+        }
+        if constexpr (M == Mode::kSwa3d) {
+          static_assert(kSplit == 2, "the 3-D window mask gives each half one t-slice");
+          if (tok_row && j < seq.nvid) {
+            const RasterGeom& g = p.rg;
+            const int kt = j / p.tile_blocks;
+            const int sb = j - kt * p.tile_blocks;
+            const int kid = seq.ids[kt];
+            const int ktw = kid % g.NW, kth = (kid / g.NW) % g.NH, ktt = kid / (g.NW * g.NH);
+            const uint64_t km = swa3d_half_mask(ktt * g.ct + sb * 2 + half, kth * g.ch,
+                                                ktw * g.cw, tws, twe);
+#pragma unroll
+            for (int c = 0; c < kCols; ++c)
+              if (!((km >> c) & 1ull)) s[c] = -INFINITY;
+            masked = true;
+          }
         }
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
 #pragma unroll

@@ -196,7 +196,7 @@ int class_video_tiles(const Geom& g, const int* w) {
 }
 
 void launch_lists(int* counts, int* ids, const Classes& cls, const Geom& g, int max_k,
-                  cudaStream_t st) {
+                  cudaStream_t st, bool token_mode = false) {
   sta::ListWindows wp;
   std::memset(&wp, 0, sizeof(wp));
   std::memcpy(wp.w, cls.win.data(), sizeof(int) * cls.win.size());
@@ -205,10 +205,36 @@ void launch_lists(int* counts, int* ids, const Classes& cls, const Geom& g, int 
   lg.NQ = g.NV + (g.has_text ? 1 : 0);
   lg.max_k = max_k;
   lg.text_block = (g.has_text && g.text_len > 0) ? 1 : 0;
+  lg.token_mode = token_mode ? 1 : 0;
+  lg.ct = g.ct; lg.ch = g.ch; lg.cw = g.cw;
   const int total = cls.nclass * lg.NQ;
   const int threads = 128;
   sta::kv_tile_list_kernel<<<(total + threads - 1) / threads, threads, 0, st>>>(
       counts, ids, wp, cls.nclass, lg);
+}
+
+// Token-window mode (3-D sliding window): key tiles covering the windows of
+// the tokens of query tile c along one axis (same rule as the list kernel).
+void token_tile_range_host(int c, int w, int cs, int n, int* s, int* e) {
+  const int X = n * cs;
+  const int we = std::min(w, X);
+  const int lo = std::max(0, std::min(c * cs - we / 2, X - we));
+  const int hi = std::max(0, std::min(c * cs + cs - 1 - we / 2, X - we));
+  *s = lo / cs;
+  *e = (hi + we - 1) / cs - *s + 1;
+}
+
+// (start, extent) of query tile t's key-tile box along the three axes.
+void tile_box(const Geom& g, const int* w, int t, bool token_mode, int st[3], int ex[3]) {
+  const int c[3] = {t / (g.NW * g.NH), (t / g.NW) % g.NH, t % g.NW};
+  const int n[3] = {g.NT, g.NH, g.NW};
+  const int cs[3] = {g.ct, g.ch, g.cw};
+  for (int a = 0; a < 3; ++a) {
+    if (token_mode)
+      token_tile_range_host(c[a], w[a], cs[a], n[a], &st[a], &ex[a]);
+    else
+      window_range_host(c[a], w[a], n[a], &st[a], &ex[a]);
+  }
 }
 
 // ------------------------------------------------------------------ workspace
@@ -246,7 +272,7 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // (text items, then by list length) and, within one length, by slice so that
 // concurrently running CTAs share K/V in L2.
 std::vector<WorkItem> plan_sta(const Geom& g, const Classes& cls, int B, int heads,
-                               int max_k, std::vector<int>* lengths) {
+                               int max_k, std::vector<int>* lengths, bool token_mode = false) {
   const int NQ = g.NV + (g.has_text ? 1 : 0);
   const int bpt = g.V / sta::kBM;
   const int text_blocks = (g.text_len + sta::kBN - 1) / sta::kBN;
@@ -259,21 +285,21 @@ std::vector<WorkItem> plan_sta(const Geom& g, const Classes& cls, int B, int hea
       const int base = slice * g.S;
       const int c = cls.head_class[h];
       const int* w = &cls.win[3 * c];
-      const int vlen = class_video_tiles(g, w) * bpt + sentinel * text_blocks;
-      std::map<int64_t, int> pending;   // start triple -> leftover block row
+      std::map<int64_t, int> pending;   // key-tile box -> leftover block row
       for (int t = 0; t < g.NV; ++t) {
+        int bs[3], be[3];
+        tile_box(g, w, t, token_mode, bs, be);
+        const int vlen = be[0] * be[1] * be[2] * bpt + sentinel * text_blocks;
         const int list = c * NQ + t;
         const int row0 = base + t * g.V;
         int qb = 0;
         for (; qb + 1 < bpt; qb += 2)
           all.push_back({vlen, slice, {row0 + qb * sta::kBM, row0 + (qb + 1) * sta::kBM, base, list}});
         if (qb < bpt) {
-          const int qw = t % g.NW, qh = (t / g.NW) % g.NH, qt = t / (g.NW * g.NH);
-          int st, sh, sw, e;
-          window_range_host(qt, w[0], g.NT, &st, &e);
-          window_range_host(qh, w[1], g.NH, &sh, &e);
-          window_range_host(qw, w[2], g.NW, &sw, &e);
-          const int64_t key = (int64_t(st) * g.NH + sh) * g.NW + sw;
+          // identical boxes give identical lists: pair the leftover blocks
+          int64_t key = 0;
+          for (int a = 0; a < 3; ++a) key = key * 4096 + bs[a];
+          for (int a = 0; a < 3; ++a) key = key * 4096 + be[a];
           auto itp = pending.find(key);
           if (itp == pending.end()) {
             pending[key] = t;
@@ -288,6 +314,9 @@ std::vector<WorkItem> plan_sta(const Geom& g, const Classes& cls, int B, int hea
       }
       for (auto& kv : pending) {
         const int t0 = kv.second;
+        int bs[3], be[3];
+        tile_box(g, w, t0, token_mode, bs, be);
+        const int vlen = be[0] * be[1] * be[2] * bpt + sentinel * text_blocks;
         all.push_back({vlen, slice, {base + t0 * g.V + (bpt - 1) * sta::kBM, -1, base, c * NQ + t0}});
       }
       if (g.has_text) {
@@ -346,7 +375,19 @@ sta_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 sta_status forward_impl(const void* q, const void* k, const void* v, void* out, float* lse,
                         int B, int heads, int d, int T, int H, int W, const int tile[3],
                         const int* window, int text_len, int has_text, void* stream,
-                        bool raster = false) {
+                        bool raster = false, const int* token_window = nullptr) {
+  // token_window != nullptr: token-level 3-D sliding window (one window of
+  // tokens for every head) instead of STA's window of tiles.
+  const bool token_mode = token_window != nullptr;
+  int tok_wins[3 * kMaxClasses];
+  if (token_mode) {
+    if (heads > kMaxClasses) return STA_ERR_UNSUPPORTED;
+    for (int a = 0; a < 3; ++a)
+      if (token_window[a] < 1) return STA_ERR_INVALID_ARG;
+    for (int h = 0; h < heads; ++h)
+      for (int a = 0; a < 3; ++a) tok_wins[3 * h + a] = token_window[a];
+    window = tok_wins;
+  }
   if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
   if (lse != nullptr && (reinterpret_cast<uintptr_t>(lse) & 3u)) return STA_ERR_INVALID_ARG;
@@ -359,6 +400,7 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (s != STA_OK) return s;
   if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
   if (g.V % sta::kBM != 0) return STA_ERR_UNSUPPORTED;
+  if (token_mode && (g.ch != 8 || g.cw != 8)) return STA_ERR_UNSUPPORTED;
   const int64_t total_rows = int64_t(B) * heads * g.S;
   if (total_rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
   // Raster order: a 128-row block of a tile must be a box {cw, bh, bt} of
@@ -382,18 +424,27 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (cls.nclass > kMaxClasses) return STA_ERR_UNSUPPORTED;
   const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
   int max_k = 1;
-  for (int c = 0; c < cls.nclass; ++c)
-    max_k = std::max(max_k, class_video_tiles(g, &cls.win[3 * c]) + sentinel);
+  for (int c = 0; c < cls.nclass; ++c) {
+    if (token_mode) {
+      for (int t = 0; t < g.NV; ++t) {
+        int bs[3], be[3];
+        tile_box(g, &cls.win[3 * c], t, true, bs, be);
+        max_k = std::max(max_k, be[0] * be[1] * be[2] + sentinel);
+      }
+    } else {
+      max_k = std::max(max_k, class_video_tiles(g, &cls.win[3 * c]) + sentinel);
+    }
+  }
   if (g.has_text) max_k = std::max(max_k, g.NV + sentinel);
   const int NQ = g.NV + (g.has_text ? 1 : 0);
   const size_t counts_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
   const size_t ids_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
 
-  const std::string key = sta_key(dev, B, heads, d, g, window);
+  const std::string key = (token_mode ? "tok:" : "") + sta_key(dev, B, heads, d, g, window);
   Workspace& ws = g_ws[dev];
   std::vector<WorkItem> fresh;
   const bool cached = (ws.plan_key == key && ws.buf != nullptr);
-  if (!cached) fresh = plan_sta(g, cls, B, heads, max_k, nullptr);
+  if (!cached) fresh = plan_sta(g, cls, B, heads, max_k, nullptr, token_mode);
   const std::vector<WorkItem>& items = cached ? ws.items : fresh;
   const size_t items_bytes = sizeof(WorkItem) * items.size();
   s = ensure_workspace(dev, counts_bytes + ids_bytes + items_bytes);
@@ -417,7 +468,7 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (s != STA_OK) return s;
 
   // a2: tile lists, rebuilt on every call.
-  launch_lists(d_counts, d_ids, cls, g, max_k, st);
+  launch_lists(d_counts, d_ids, cls, g, max_k, st, token_mode);
   STA_CUDA_TRY(cudaGetLastError());
 
   FwdParams prm;
@@ -439,6 +490,9 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   prm.rg.ct = g.ct; prm.rg.ch = g.ch; prm.rg.cw = g.cw;
   prm.rg.H = g.H; prm.rg.W = g.W;
   prm.rg.NH = g.NH; prm.rg.NW = g.NW;
+  prm.rg.T = g.T;
+  if (token_mode)
+    for (int a = 0; a < 3; ++a) prm.win3[a] = token_window[a];
   if (raster) {
     CUtensorMap q5, k5, v5;
     const int slices = B * heads;
@@ -446,10 +500,17 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
     if (s == STA_OK) s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
     if (s == STA_OK) s = make_raster_map(&v5, v, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
     if (s != STA_OK) return s;
+    if (token_mode) {
+      if (d == 128)
+        return launch_attn<128, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5,
+                                                     &v5);
+      return launch_attn<64, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
+    }
     if (d == 128)
       return launch_attn<128, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
     return launch_attn<64, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
   }
+  if (token_mode) return STA_ERR_UNSUPPORTED;
   if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
   return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
 }
@@ -705,6 +766,15 @@ sta_status sta_forward_raster(const void* q, const void* k, const void* v, void*
                               void* stream) {
   return forward_impl(q, k, v, out, lse, B, heads, d, T, H, W, tile, window, text_len,
                       has_text, stream, true);
+}
+
+sta_status sta_swa3d_forward(const void* q, const void* k, const void* v, void* out, int B,
+                             int heads, int d, int T, int H, int W, const int tile[3],
+                             const int window_tokens[3], int text_len, int has_text,
+                             void* stream) {
+  if (window_tokens == nullptr) return STA_ERR_INVALID_ARG;
+  return forward_impl(q, k, v, out, nullptr, B, heads, d, T, H, W, tile, window_tokens,
+                      text_len, has_text, stream, true, window_tokens);
 }
 
 sta_status sta_forward_noalloc(const void* q, const void* k, const void* v, void* out, int B,

@@ -28,6 +28,8 @@ struct ListGeom {
   int NQ;          // rows per window class (NV, or NV + 1 with text)
   int max_k;
   int text_block;  // 1 when the text block has valid keys
+  int token_mode;  // windows counted in tokens (3-D sliding window), not tiles
+  int ct, ch, cw;  // tile size (token mode)
 };
 
 __device__ __forceinline__ void window_range(int c, int w, int n, int& s,
@@ -36,6 +38,22 @@ __device__ __forceinline__ void window_range(int c, int w, int n, int& s,
   s = c - e / 2;
   if (s < 0) s = 0;
   if (s > n - e) s = n - e;
+}
+
+// Token-window mode: the key tiles that hold any key of the windows of the
+// tokens of query tile c along one axis.  Token windows are centred on the
+// token and shifted inward at the border; their starts grow with the token,
+// so the first and last token of the tile bound the union.
+__device__ __forceinline__ void token_tile_range(int c, int w, int cs, int n, int& s,
+                                                 int& e) {
+  const int X = n * cs;
+  const int we = w < X ? w : X;
+  int lo = c * cs - we / 2;
+  lo = lo < 0 ? 0 : (lo > X - we ? X - we : lo);
+  int hi = c * cs + cs - 1 - we / 2;
+  hi = hi < 0 ? 0 : (hi > X - we ? X - we : hi);
+  s = lo / cs;
+  e = (hi + we - 1) / cs - s + 1;
 }
 
 // One thread per (class, row).
@@ -53,9 +71,15 @@ __global__ void __launch_bounds__(128) kv_tile_list_kernel(
     const int qh = (row / g.NW) % g.NH;
     const int qt = row / (g.NW * g.NH);
     int st, et, sh, eh, sw, ew;
-    window_range(qt, windows.w[cls * 3 + 0], g.NT, st, et);
-    window_range(qh, windows.w[cls * 3 + 1], g.NH, sh, eh);
-    window_range(qw, windows.w[cls * 3 + 2], g.NW, sw, ew);
+    if (g.token_mode) {
+      token_tile_range(qt, windows.w[cls * 3 + 0], g.ct, g.NT, st, et);
+      token_tile_range(qh, windows.w[cls * 3 + 1], g.ch, g.NH, sh, eh);
+      token_tile_range(qw, windows.w[cls * 3 + 2], g.cw, g.NW, sw, ew);
+    } else {
+      window_range(qt, windows.w[cls * 3 + 0], g.NT, st, et);
+      window_range(qh, windows.w[cls * 3 + 1], g.NH, sh, eh);
+      window_range(qw, windows.w[cls * 3 + 2], g.NW, sw, ew);
+    }
     for (int t = st; t < st + et; ++t)
       for (int h = sh; h < sh + eh; ++h)
         for (int w = sw; w < sw + ew; ++w) out[n++] = (t * g.NH + h) * g.NW + w;

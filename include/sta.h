@@ -143,6 +143,26 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v,
                            void* out, int B, int hq, int hkv, int d, int S,
                            int window, int causal, void* stream);
 
+/*
+ * sta_swa3d_forward - token-level 3-D sliding-window attention, the
+ * mixed-block baseline that README "Why is STA Fast?" compares STA with
+ * ("2D/3D Sliding Window Attention (SWA) creates many mixed blocks").  Every
+ * video query token attends to the keys of a window of
+ * window_tokens = (Wt, Wh, Ww) TOKENS centred on it and shifted inward at the
+ * grid border (clipped to the grid), plus the first text_len text keys; text
+ * queries attend to every video key and the first text_len text keys.
+ *   q, k, v, out: [B, heads, S, d] bf16 device, RASTER order (as
+ *   sta_forward_raster); one window for all heads (HOST int32[3]).
+ * The key tiles of a query tile are those holding any key of its tokens'
+ * windows; every video block is masked per element.  Requires tiles with
+ * ch = cw = 8 and ct even, d in {64,128}, else STA_ERR_UNSUPPORTED.
+ */
+sta_status sta_swa3d_forward(const void* q, const void* k, const void* v,
+                             void* out, int B, int heads, int d, int T, int H,
+                             int W, const int tile[3],
+                             const int window_tokens[3], int text_len,
+                             int has_text, void* stream);
+
 /* Synchronises `stream`, returns STA_ERR_DEVICE_TIMEOUT if any kernel of this
  * library recorded a gave-up wait since the last call (and clears it), else
  * STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
