@@ -224,6 +224,7 @@ def run_ours(args):
 
     import block_sparse_local_b200 as sta
     from block_sparse_local_b200 import workloads
+    from block_sparse_local_b200.dist_timing import max_over_ranks, rank_seed
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -246,7 +247,7 @@ def run_ours(args):
     gq = torch.Generator(device=dev)
     qkv = []
     for i in range(3):
-        gq.manual_seed(w.seed * 1000 + i + 17 * rank)
+        gq.manual_seed(rank_seed(w.seed * 1000 + i, rank))
         qkv.append(torch.randn((w.B, w.heads, w.S, w.d), generator=gq, device=dev,
                                dtype=torch.float32).to(torch.bfloat16))
     q, k, v = qkv
@@ -288,10 +289,7 @@ def run_ours(args):
     sta.device_status(dev)
     ms = t0.elapsed_time(t1) / args.steps
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
-    if world > 1:
-        tt = torch.tensor([ms, attn_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, attn_ms = float(tt[0]), float(tt[1])
+    ms, attn_ms = max_over_ranks([ms, attn_ms], device=dev)
     value = world * flops / (ms * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers
@@ -317,10 +315,7 @@ def run_ours(args):
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt[0])
+        (e2e_ms,) = max_over_ranks([e2e_ms], device=dev)
         nbytes = q.numel() * q.element_size()
         e2e = {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                "ms_per_step": e2e_ms, "h2d_bytes_per_step": 3 * nbytes,

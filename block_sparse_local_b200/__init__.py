@@ -30,7 +30,7 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
             "sta_device_status", "sta_status_string", "sta_shutdown",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
-            "sta_swa3d_forward")
+            "sta_swa3d_forward", "sta_debug_inject")
 
 
 class StaError(RuntimeError):
@@ -70,6 +70,7 @@ def lib():
     L.sta_swa3d_forward.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
+    L.sta_debug_inject.argtypes = [_I, _I]
     L.sta_status_string.argtypes = [_I]
     L.sta_status_string.restype = ctypes.c_char_p
     L.sta_shutdown.argtypes = []

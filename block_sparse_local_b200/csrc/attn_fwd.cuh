@@ -349,11 +349,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0 && !skip) {
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
-      mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
-      for (int s = 0; s < (two ? 2 : 1); ++s) {
-        const int qrow = s ? item.q1 : item.q0;
-        load_block<D, R>(smem + C::kQOff + s * C::kBlockBytes, &tmap_q, &tmap_q5, q_full, qrow,
-                         p, pol_q);
+      const bool drop_q = *reinterpret_cast<volatile int*>(&g_inject) == 1;
+      if (!drop_q) {
+        mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
+        for (int s = 0; s < (two ? 2 : 1); ++s) {
+          const int qrow = s ? item.q1 : item.q0;
+          load_block<D, R>(smem + C::kQOff + s * C::kBlockBytes, &tmap_q, &tmap_q5, q_full,
+                           qrow, p, pol_q);
+        }
       }
       int issued = 0;
       for (int j = 0; j < n; ++j) {
@@ -374,7 +377,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         issued = j * 2 + 2;
       }
       // Leave no copy in flight: wait for the last load of every stage.
-      mbar_wait_drain(q_full, 0);
+      if (!drop_q) mbar_wait_drain(q_full, 0);
       const int nk = (issued + 1) / 2, nv = issued / 2;
       for (int s = 0; s < KST && s < nk; ++s) {
         const int last = s + ((nk - 1 - s) / KST) * KST;

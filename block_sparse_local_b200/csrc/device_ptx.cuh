@@ -1,8 +1,8 @@
 // device_ptx.cuh - thin inline-PTX wrappers for sm_100a: mbarriers with
 // bounded waits, TMA tile loads, tcgen05 (TMEM alloc, MMA, commit, ld/st).
 //
-// Every wait in this library is bounded: after kWaitLimitNs of polling (or as
-// soon as another CTA or warp has given up) it returns false, the caller
+// Every wait in this library is bounded: after g_wait_limit_ns of polling (or
+// as soon as another CTA or warp has given up) it returns false, the caller
 // records STA_ERR_DEVICE_TIMEOUT in the device error word and unwinds.
 #pragma once
 
@@ -15,7 +15,13 @@ namespace sta {
 // Device error word (bit 0: a wait gave up).  One per process.
 __device__ unsigned int g_error_word = 0;
 
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s for a single wait
+// Time limit of a single wait (2 s; lowered only by the fault-injection hook).
+__device__ unsigned long long g_wait_limit_ns = 2000000000ull;
+
+// Fault injection for tests (sta_debug_inject): 1 = the attention kernel's
+// producer does not load Q, so the MMA warp waits on an arrival that never
+// comes and the bounded-wait path runs.
+__device__ int g_inject = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -87,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 255u) == 0u) {
       if (*abort != 0 || error_raised()) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > *reinterpret_cast<volatile unsigned long long*>(&g_wait_limit_ns)) {
         raise_error(1u);
         *abort = 1;
         return false;

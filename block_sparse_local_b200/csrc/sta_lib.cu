@@ -844,6 +844,15 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   return launch_attn<64, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
 }
 
+sta_status sta_debug_inject(int mode, int wait_limit_ms) {
+  if (mode < 0 || mode > 1 || wait_limit_ms < 1) return STA_ERR_INVALID_ARG;
+  const unsigned long long limit = static_cast<unsigned long long>(wait_limit_ms) * 1000000ull;
+  STA_CUDA_TRY(cudaDeviceSynchronize());
+  STA_CUDA_TRY(cudaMemcpyToSymbol(sta::g_inject, &mode, sizeof(mode)));
+  STA_CUDA_TRY(cudaMemcpyToSymbol(sta::g_wait_limit_ns, &limit, sizeof(limit)));
+  return STA_OK;
+}
+
 sta_status sta_device_status(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return STA_ERR_CUDA;

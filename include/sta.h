@@ -168,6 +168,18 @@ sta_status sta_swa3d_forward(const void* q, const void* k, const void* v,
  * STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
 sta_status sta_device_status(void* stream);
 
+/*
+ * sta_debug_inject - fault injection for tests; no passage of the pages
+ * corresponds to it.  mode 1: the attention kernel's TMA producer skips the
+ * Q load, so the MMA warp waits for an arrival that never comes; the bounded
+ * wait gives up after wait_limit_ms, the kernel drains its in-flight copies,
+ * frees its tensor memory and exits, and sta_device_status() reports
+ * STA_ERR_DEVICE_TIMEOUT.  mode 0 with wait_limit_ms = 2000 restores normal
+ * operation.  Synchronises the current device; applies to every later launch
+ * on it.  No GPU fault, trap or hang is involved.
+ */
+sta_status sta_debug_inject(int mode, int wait_limit_ms);
+
 /* Static, never NULL. */
 const char* sta_status_string(sta_status s);
 
