@@ -400,6 +400,36 @@ def run_ours(args):
                                    "sta_speedup": s3_ms / ms}}
         del sq, sk, sv, so, m_q, m_k, m_v, m_o
 
+        # Hilbert-order vs raster-order block-sparse 2-D slide attention on the
+        # 2-D image workload's shape (256 x 256 tokens, 8 x 16 heads, d=64),
+        # 21 x 21 token window; inputs already in each order.
+        iw = workloads.IMAGE_2D
+        n2, w2 = iw.W, 21
+        hq, hk, hv = workloads.sta_inputs(iw, device=dev)
+        ho = torch.empty_like(hq)
+        pairs2 = iw.B * iw.heads * n2 * n2 * w2 * w2
+        hil = {"workload": f"image2d_{n2}x{n2}_slide{w2}", "window": w2}
+        for order in ("raster", "hilbert"):
+            counts, ids, cls = sta.build_slide_block_lists(n2, w2, order, device=dev)
+            nonempty = int(counts.sum())
+            partial = int((cls == 1).sum())
+            for _ in range(2):
+                sta.slide2d_forward(hq, hk, hv, n2, w2, order, out=ho)
+            torch.cuda.synchronize(dev)
+            a.record(stream)
+            for _ in range(5):
+                sta.slide2d_forward(hq, hk, hv, n2, w2, order, out=ho)
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            t2 = a.elapsed_time(b) / 5
+            hil[order] = {"ms": t2, "effective_tflops": 4.0 * iw.d * pairs2 / (t2 * 1e-3) / 1e12,
+                          "nonempty_blocks": nonempty, "partial_blocks": partial,
+                          "full_blocks": nonempty - partial}
+        hil["hilbert_speedup"] = hil["raster"]["ms"] / hil["hilbert"]["ms"]
+        sta.device_status(dev)
+        swa["hilbert_slide2d"] = hil
+        del hq, hk, hv, ho
+
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (attn_ms * 1e-3) / 1e12

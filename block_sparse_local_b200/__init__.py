@@ -21,6 +21,7 @@ __all__ = [
     "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
     "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
+    "hilbert_reorder", "build_slide_block_lists", "slide2d_forward", "slide_attention_2d",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -30,7 +31,8 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
             "sta_device_status", "sta_status_string", "sta_shutdown",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
-            "sta_swa3d_forward", "sta_debug_inject")
+            "sta_swa3d_forward", "sta_debug_inject", "sta_hilbert_reorder",
+            "sta_build_slide_block_lists", "sta_slide2d_forward")
 
 
 class StaError(RuntimeError):
@@ -71,6 +73,9 @@ def lib():
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_debug_inject.argtypes = [_I, _I]
+    L.sta_hilbert_reorder.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P]
+    L.sta_build_slide_block_lists.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P]
+    L.sta_slide2d_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
     L.sta_status_string.argtypes = [_I]
     L.sta_status_string.restype = ctypes.c_char_p
     L.sta_shutdown.argtypes = []
@@ -243,6 +248,52 @@ def swa3d_forward(q, k, v, window_tokens, text_length, has_text, video_shape,
                                    _I3(*tile), _I3(*window_tokens), int(text_length),
                                    int(has_text), _stream(q)), "sta_swa3d_forward")
     return out
+
+
+ORDERS = {"raster": 0, "hilbert": 1}
+
+
+def hilbert_reorder(x, n, to_hilbert=True, out=None):
+    """[B, heads, n*n, d] rows between raster and Hilbert order (bit-exact)."""
+    _check_qkv(x)
+    out = torch.empty_like(x) if out is None else out
+    B, nh, _, d = x.shape
+    _check(lib().sta_hilbert_reorder(_ptr(x), _ptr(out), B, nh, d, n, int(to_hilbert),
+                                     _stream(x)), "sta_hilbert_reorder")
+    return out
+
+
+def build_slide_block_lists(n, window, order="hilbert", device="cuda"):
+    """(counts [nb], ids [nb, nb], classes [nb, nb]) of 2-D slide attention."""
+    nb = n * n // 128
+    counts = torch.empty(nb, dtype=torch.int32, device=device)
+    ids = torch.empty((nb, nb), dtype=torch.int32, device=device)
+    cls = torch.empty((nb, nb), dtype=torch.int32, device=device)
+    _check(lib().sta_build_slide_block_lists(_ptr(counts), _ptr(ids), _ptr(cls), nb, n,
+                                             int(window), ORDERS[order], _stream(counts)),
+           "sta_build_slide_block_lists")
+    return counts, ids, cls
+
+
+def slide2d_forward(q, k, v, n, window, order="hilbert", out=None):
+    """Block-sparse 2-D slide attention on q, k, v stored in `order`."""
+    _check_qkv(q, k, v)
+    B, nh, _, d = q.shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib().sta_slide2d_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d, n,
+                                     int(window), ORDERS[order], _stream(q)),
+           "sta_slide2d_forward")
+    return out
+
+
+def slide_attention_2d(q, k, v, n, window, order="hilbert"):
+    """Raster-ordered in and out; with order='hilbert' the tokens are reordered
+    along the Hilbert curve, attended block-sparsely, and put back."""
+    if order == "raster":
+        return slide2d_forward(q, k, v, n, window, "raster")
+    qh, kh, vh = (hilbert_reorder(x, n, True) for x in (q, k, v))
+    oh = slide2d_forward(qh, kh, vh, n, window, "hilbert")
+    return hilbert_reorder(oh, n, False)
 
 
 def swa_forward(q, k, v, window, causal=True, out=None):

@@ -53,7 +53,7 @@ constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
 constexpr int kWarpSoftmax0 = 2;
 
-enum class Mode { kSta = 0, kSwa = 1, kSwa3d = 2 };
+enum class Mode { kSta = 0, kSwa = 1, kSwa3d = 2, kSlide2d = 3 };
 
 struct WorkItem {
   int q0;       // first row (in the [B*heads*S, d] view) of query block 0
@@ -87,6 +87,9 @@ struct FwdParams {
   int text_sentinel;  // lists end with the text block
   int window;         // kSwa: tokens
   int win3[3];        // kSwa3d: (Wt, Wh, Ww) token window
+  const uint32_t* coords;  // kSlide2d: x | y << 16 of every position of the order
+  int grid_n;         // kSlide2d: n of the n x n grid
+  int win2;           // kSlide2d: w of the w x w window
   float scale_log2;   // log2(e) / sqrt(d)
   __nv_bfloat16* out;
   float* lse;
@@ -510,6 +513,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
       }
       (void)tok_row;
+      // kSlide2d: this query's w x w window
+      int sxlo = 0, sylo = 0, swe = 0;
+      if constexpr (M == Mode::kSlide2d) {
+        const int qpos = (slot ? item.q1 : item.q0) + r - item.kv_base;
+        const uint32_t qc = p.coords[qpos];
+        swe = p.win2 < p.grid_n ? p.win2 : p.grid_n;
+        sxlo = static_cast<int>(qc & 0xffff) - swe / 2;
+        sxlo = sxlo < 0 ? 0 : (sxlo > p.grid_n - swe ? p.grid_n - swe : sxlo);
+        sylo = static_cast<int>(qc >> 16) - swe / 2;
+        sylo = sylo < 0 ? 0 : (sylo > p.grid_n - swe ? p.grid_n - swe : sylo);
+      }
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
@@ -528,6 +542,24 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int c = 0; c < kCols; ++c)
             if (c < lo || c >= hi) s[c] = -INFINITY;
+        }
+        if constexpr (M == Mode::kSlide2d) {
+          // per-element 2-D window test against the keys' grid coordinates
+          const uint4* kc = reinterpret_cast<const uint4*>(
+              p.coords + static_cast<size_t>(seq.ids[j]) * kBN + half * kCols);
+#pragma unroll
+          for (int c4 = 0; c4 < kCols / 4; ++c4) {
+            const uint4 v4 = __ldg(kc + c4);
+            const uint32_t cv[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t dx = (cv[e] & 0xffffu) - static_cast<uint32_t>(sxlo);
+              const uint32_t dy = (cv[e] >> 16) - static_cast<uint32_t>(sylo);
+              if (dx >= static_cast<uint32_t>(swe) || dy >= static_cast<uint32_t>(swe))
+                s[c4 * 4 + e] = -INFINITY;
+            }
+          }
+          masked = true;
         }
         if constexpr (M == Mode::kSwa3d) {
           static_assert(kSplit == 2, "the 3-D window mask gives each half one t-slice");

@@ -20,6 +20,7 @@
 #include "reorder.cuh"
 #include "tile_lists.cuh"
 #include "attn_fwd.cuh"
+#include "hilbert.cuh"
 
 namespace {
 
@@ -694,6 +695,53 @@ sta_status forward_noalloc_impl(const void* q, const void* k, const void* v, voi
   return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
 }
 
+// ------------------------------------------------------------------ 2-D slide
+// Workspace of the 2-D slide-attention path (coordinate table, block
+// rectangles, pair lists and plan), separate from the STA workspace.
+struct Slide2dWs {
+  void* buf = nullptr;
+  size_t cap = 0;
+  std::string key;
+};
+Slide2dWs g_ws2d[64];
+
+int ilog2_exact(int n) {
+  int l = 0;
+  while ((1 << l) < n) ++l;
+  return (1 << l) == n ? l : -1;
+}
+
+sta_status slide2d_check(int n, int window, int order) {
+  const int l = ilog2_exact(n);
+  if (l < 4 || l > 15) return STA_ERR_UNSUPPORTED;  // 16 <= n <= 32768, power of two
+  if (window < 1) return STA_ERR_INVALID_ARG;
+  if (order != 0 && order != 1) return STA_ERR_INVALID_ARG;
+  if (order == 0 && n < 128) return STA_ERR_UNSUPPORTED;  // raster blocks must be row pieces
+  return STA_OK;
+}
+
+sta_status slide2d_ensure(int dev, size_t bytes) {
+  Slide2dWs& w = g_ws2d[dev];
+  if (w.cap >= bytes) return STA_OK;
+  if (w.buf) {
+    STA_CUDA_TRY(cudaFree(w.buf));
+    w.buf = nullptr;
+    w.cap = 0;
+  }
+  STA_CUDA_TRY(cudaMalloc(&w.buf, bytes));
+  w.cap = bytes;
+  w.key.clear();
+  return STA_OK;
+}
+
+// coords + rects for `order` into the given device buffers.
+void launch_coords_rects(uint32_t* coords, int4* rects, int n, int order, cudaStream_t st) {
+  const int l = ilog2_exact(n);
+  const int N = n * n, nb = N / 128;
+  sta::order_coords_kernel<<<(N + 255) / 256, 256, 0, st>>>(coords, l, order);
+  sta::block_rect_kernel<<<(nb * 32 + 255) / 256, 256, 0, st>>>(coords, rects, nb);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -853,6 +901,134 @@ sta_status sta_debug_inject(int mode, int wait_limit_ms) {
   return STA_OK;
 }
 
+sta_status sta_hilbert_reorder(const void* in, void* out, int B, int heads, int d, int n,
+                               int to_hilbert, void* stream) {
+  if (!in || !out || in == out || !aligned16(in) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1 || d < 1 || (to_hilbert != 0 && to_hilbert != 1)) return STA_ERR_INVALID_ARG;
+  const int l = ilog2_exact(n);
+  if (l < 1 || l > 15) return STA_ERR_UNSUPPORTED;
+  if ((d * 2) % 16 != 0) return STA_ERR_UNSUPPORTED;
+  const int vec = d * 2 / 16;
+  if (vec != 4 && vec != 8 && vec != 16 && vec != 32) return STA_ERR_UNSUPPORTED;
+  int dev = 0;
+  sta_status s = current_device(&dev);
+  if (s != STA_OK) return s;
+  const long long total = static_cast<long long>(B) * heads * n * n * vec;
+  const int grid = static_cast<int>(std::min<long long>((total + 255) / 256, 148LL * 64));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint4* a = static_cast<const uint4*>(in);
+  uint4* b = static_cast<uint4*>(out);
+  switch (vec) {
+    case 4: sta::hilbert_permute_kernel<4><<<grid, 256, 0, st>>>(a, b, l, total, to_hilbert); break;
+    case 8: sta::hilbert_permute_kernel<8><<<grid, 256, 0, st>>>(a, b, l, total, to_hilbert); break;
+    case 16: sta::hilbert_permute_kernel<16><<<grid, 256, 0, st>>>(a, b, l, total, to_hilbert); break;
+    default: sta::hilbert_permute_kernel<32><<<grid, 256, 0, st>>>(a, b, l, total, to_hilbert); break;
+  }
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status sta_build_slide_block_lists(int* counts, int* ids, int* classes, int max_k, int n,
+                                       int window, int order, void* stream) {
+  if (!counts || !ids) return STA_ERR_INVALID_ARG;
+  sta_status s = slide2d_check(n, window, order);
+  if (s != STA_OK) return s;
+  const int nb = n * n / 128;
+  if (max_k < nb) return STA_ERR_INVALID_ARG;
+  if (nb > 8192) return STA_ERR_UNSUPPORTED;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  std::lock_guard<std::mutex> lock(g_mu);
+  const size_t cbytes = align_up(sizeof(uint32_t) * size_t(n) * n, 256);
+  s = slide2d_ensure(dev, cbytes + sizeof(int4) * nb);
+  if (s != STA_OK) return s;
+  g_ws2d[dev].key.clear();
+  uint8_t* w = static_cast<uint8_t*>(g_ws2d[dev].buf);
+  uint32_t* coords = reinterpret_cast<uint32_t*>(w);
+  int4* rects = reinterpret_cast<int4*>(w + cbytes);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  launch_coords_rects(coords, rects, n, order, st);
+  const size_t smem = sizeof(int) * (512 + nb);
+  sta::slide_block_list_kernel<<<nb, 256, smem, st>>>(counts, ids, classes, max_k, coords, rects,
+                                                      nb, n, window, 1);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void* out, int B,
+                               int heads, int d, int n, int window, int order, void* stream) {
+  if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out)) return STA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v || B < 1 || heads < 1) return STA_ERR_INVALID_ARG;
+  sta_status s = slide2d_check(n, window, order);
+  if (s != STA_OK) return s;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  const int N = n * n, nb = N / 128, np = nb / 2;
+  if (nb > 8192) return STA_ERR_UNSUPPORTED;
+  const int64_t rows = int64_t(B) * heads * N;
+  if (rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t cbytes = align_up(sizeof(uint32_t) * size_t(N), 256);
+  const size_t rbytes = align_up(sizeof(int4) * size_t(nb), 256);
+  const size_t nbytes = align_up(sizeof(int) * size_t(np), 256);
+  const size_t ibytes = align_up(sizeof(int) * size_t(np) * nb, 256);
+  const size_t pbytes = sizeof(WorkItem) * size_t(B) * heads * np;
+  s = slide2d_ensure(dev, cbytes + rbytes + nbytes + ibytes + pbytes);
+  if (s != STA_OK) return s;
+  Slide2dWs& ws = g_ws2d[dev];
+  uint8_t* w = static_cast<uint8_t*>(ws.buf);
+  uint32_t* coords = reinterpret_cast<uint32_t*>(w);
+  int4* rects = reinterpret_cast<int4*>(w + cbytes);
+  int* counts = reinterpret_cast<int*>(w + cbytes + rbytes);
+  int* ids = reinterpret_cast<int*>(w + cbytes + rbytes + nbytes);
+  WorkItem* items = reinterpret_cast<WorkItem*>(w + cbytes + rbytes + nbytes + ibytes);
+  const std::string key = "s2d:" + std::to_string(B) + ":" + std::to_string(heads) + ":" +
+                          std::to_string(n) + ":" + std::to_string(order);
+  if (ws.key != key) {
+    std::vector<WorkItem> plan;
+    plan.reserve(size_t(B) * heads * np);
+    for (int sl = 0; sl < B * heads; ++sl)
+      for (int pi = 0; pi < np; ++pi)
+        plan.push_back({sl * N + 2 * pi * 128, sl * N + (2 * pi + 1) * 128, sl * N, pi});
+    STA_CUDA_TRY(cudaMemcpyAsync(items, plan.data(), sizeof(WorkItem) * plan.size(),
+                                 cudaMemcpyHostToDevice, st));
+    ws.key = key;
+  }
+  // key-block lists of query-block pairs (union), rebuilt on every call
+  launch_coords_rects(coords, rects, n, order, st);
+  sta::slide_block_list_kernel<<<np, 256, sizeof(int) * (512 + nb), st>>>(
+      counts, ids, nullptr, nb, coords, rects, nb, n, window, 2);
+  STA_CUDA_TRY(cudaGetLastError());
+  CUtensorMap mq, mk, mv;
+  s = make_row_map(&mq, q, rows, d);
+  if (s == STA_OK) s = make_row_map(&mk, k, rows, d);
+  if (s == STA_OK) s = make_row_map(&mv, v, rows, d);
+  if (s != STA_OK) return s;
+  FwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.items = items;
+  prm.counts = counts;
+  prm.ids = ids;
+  prm.max_k = nb;
+  prm.tile_blocks = 1;
+  prm.V = 128;
+  prm.L_v = N;
+  prm.coords = coords;
+  prm.grid_n = n;
+  prm.win2 = window;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  const int num_items = B * heads * np;
+  if (d == 128) return launch_attn<128, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
+  return launch_attn<64, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
+}
+
 sta_status sta_device_status(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return STA_ERR_CUDA;
@@ -876,6 +1052,11 @@ void sta_shutdown(void) {
       cudaSetDevice(i);
       cudaFree(g_ws[i].buf);
       g_ws[i] = Workspace();
+    }
+    if (g_ws2d[i].buf != nullptr) {
+      cudaSetDevice(i);
+      cudaFree(g_ws2d[i].buf);
+      g_ws2d[i] = Slide2dWs();
     }
   }
   cudaSetDevice(dev);

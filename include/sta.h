@@ -163,6 +163,44 @@ sta_status sta_swa3d_forward(const void* q, const void* k, const void* v,
                              const int window_tokens[3], int text_len,
                              int has_text, void* stream);
 
+/*
+ * Hilbert-order 2-D local attention ("Hilbert-guided block-sparse local
+ * attention" blog page): image tokens of an n x n grid (n a power of two,
+ * 16 <= n <= 32768) are reordered along a Hilbert curve so that 2-D windows
+ * become contiguous runs; block-sparse slide attention then skips more
+ * (empty) blocks and masks fewer (partial) ones than in row-by-row order.
+ * Curve: recursive quadrant rotation, starting at (0,0), ending at (n-1,0).
+ * Slide window: w x w tokens centred on the query, shifted inward at the
+ * border.  order: 0 raster (y*n + x; needs n >= 128 so that 128-token blocks
+ * are row pieces), 1 Hilbert.
+ *
+ * sta_hilbert_reorder - [B, heads, n*n, d] bf16 rows, raster -> Hilbert order
+ * (to_hilbert = 1: out[pos] = in[raster(pos)]) or back (0).  Bit-exact.
+ */
+sta_status sta_hilbert_reorder(const void* in, void* out, int B, int heads,
+                               int d, int n, int to_hilbert, void* stream);
+
+/*
+ * sta_build_slide_block_lists - for each 128-token query block (in `order`),
+ * the ascending key blocks holding at least one allowed key, and their class
+ * (1 partial, 2 full: every pair of the block allowed), exact; unused slots
+ * -1 / 0.  counts: device int32 [nb], ids / classes: device int32
+ * [nb][max_k], nb = n*n/128, max_k >= nb (classes may be NULL).
+ */
+sta_status sta_build_slide_block_lists(int* counts, int* ids, int* classes,
+                                       int max_k, int n, int window, int order,
+                                       void* stream);
+
+/*
+ * sta_slide2d_forward - block-sparse slide attention on q, k, v, out
+ * [B, heads, n*n, d] bf16 stored in `order`; each pair of consecutive query
+ * blocks runs over the union of their key blocks with a per-element window
+ * mask (every non-empty block is treated as partial).  d in {64,128}.
+ */
+sta_status sta_slide2d_forward(const void* q, const void* k, const void* v,
+                               void* out, int B, int heads, int d, int n,
+                               int window, int order, void* stream);
+
 /* Synchronises `stream`, returns STA_ERR_DEVICE_TIMEOUT if any kernel of this
  * library recorded a gave-up wait since the last call (and clears it), else
  * STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
