@@ -430,6 +430,29 @@ def run_ours(args):
         swa["hilbert_slide2d"] = hil
         del hq, hk, hv, ho
 
+        # backward pass of the same STA workload (tile order): dQ, dK, dV from
+        # the saved LSE; algorithmic work 5 matmuls of 2*d per retained pair
+        qt, kt, vt = (sta.tile_reorder(x, shape, w.tile, w.has_text) for x in (q, k, v))
+        ot, lset = sta.forward(qt, kt, vt, w.windows, w.text_len, w.has_text, shape, w.tile,
+                               return_lse=True)
+        dot = torch.randn_like(qt, dtype=torch.float32).to(torch.bfloat16)
+        for _ in range(2):
+            sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape,
+                         w.tile)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(3):
+            sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape,
+                         w.tile)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        bms = a.elapsed_time(b) / 3
+        sta.device_status(dev)
+        swa["backward"] = {"workload": w.name, "ms": bms,
+                           "effective_tflops": 10.0 * w.d * pairs / (bms * 1e-3) / 1e12,
+                           "flop_model": "10*d per retained pair (5 matmuls)"}
+        del qt, kt, vt, ot, lset, dot
+
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (attn_ms * 1e-3) / 1e12

@@ -22,6 +22,7 @@ __all__ = [
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
     "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
     "hilbert_reorder", "build_slide_block_lists", "slide2d_forward", "slide_attention_2d",
+    "backward", "SlidingTileAttentionFunction",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -32,7 +33,7 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_device_status", "sta_status_string", "sta_shutdown",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
             "sta_swa3d_forward", "sta_debug_inject", "sta_hilbert_reorder",
-            "sta_build_slide_block_lists", "sta_slide2d_forward")
+            "sta_build_slide_block_lists", "sta_slide2d_forward", "sta_backward")
 
 
 class StaError(RuntimeError):
@@ -73,6 +74,7 @@ def lib():
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_debug_inject.argtypes = [_I, _I]
+    L.sta_backward.argtypes = [_P] * 9 + fwd
     L.sta_hilbert_reorder.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P]
     L.sta_build_slide_block_lists.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P]
     L.sta_slide2d_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]
@@ -211,6 +213,39 @@ def forward_raster(q, k, v, window_size, text_length, has_text, video_shape,
                                     _I3(*tile), _windows(window_size, nh), int(text_length),
                                     int(has_text), _stream(q)), "sta_forward_raster")
     return (out, lse) if return_lse else out
+
+
+def backward(q, k, v, out, dout, lse, window_size, text_length, has_text, video_shape,
+             tile=(6, 8, 8)):
+    """Gradients (dq, dk, dv) of forward() on TILE-ordered tensors; lse from
+    forward(..., return_lse=True)."""
+    _check_qkv(q, k, v, out, dout)
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    dq, dk, dv = (torch.empty_like(q) for _ in range(3))
+    _check(lib().sta_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, nh, d, T, H, W, _I3(*tile),
+                              _windows(window_size, nh), int(text_length), int(has_text),
+                              _stream(q)), "sta_backward")
+    return dq, dk, dv
+
+
+class SlidingTileAttentionFunction(torch.autograd.Function):
+    """Differentiable STA on TILE-ordered q, k, v (forward keeps the LSE)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, window_size, text_length, has_text, video_shape, tile):
+        out, lse = forward(q, k, v, window_size, text_length, has_text, video_shape, tile,
+                           return_lse=True)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.args = (window_size, text_length, has_text, video_shape, tile)
+        return out
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, out, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, out, dout.contiguous(), lse, *ctx.args)
+        return dq, dk, dv, None, None, None, None, None
 
 
 def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,

@@ -1,0 +1,409 @@
+// attn_bwd.cuh - STA backward pass for sm_100a (dQ, dK, dV from the saved
+// log-sum-exp of the forward).
+//
+// The STA pages give the forward only; the backward is the gradient of that
+// function.  With S = Q K^T / sqrt(d) on allowed pairs, P = softmax(S),
+// D_i = sum_c dO_ic O_ic:  dP = dO V^T,  dS = P (dP - D),
+// dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),  dV = P^T dO.
+//
+// Two kernels share one template, one 128-row block per CTA:
+//  * kDKV = false (dQ): resident Q, dO; streams the query block's key
+//    blocks (the forward's tile lists).  TMEM: S [0,128), dP [128,256),
+//    dQ accumulator [256, 256+d).
+//  * kDKV = true (dK, dV): resident K, V of one key block; streams the query
+//    blocks whose windows hold that key tile (transposed tile lists), with
+//    their log2-domain LSE and D.  TMEM: S^T [0,128), dP^T [128,256),
+//    dV [256,256+d), dK [256+d, 256+2d).
+// Warps: 0 TMA producer, 1 MMA issuer (S and dP by SS tcgen05.mma, then the
+// accumulators by TS tcgen05.mma with P / dS from TMEM), 2-9 elementwise:
+// two warps per TMEM lane quarter, 64 columns each.  A warp writes its packed
+// bf16 P / dS into the first 32 of its own 64 columns, so no warp overwrites
+// scores another warp still has to read; the accumulate MMAs take the two
+// halves as two K ranges.
+#pragma once
+
+#include "device_ptx.cuh"
+#include "attn_fwd.cuh"
+
+namespace sta {
+
+constexpr int kBwdThreads = 320;
+
+struct BwdParams {
+  const WorkItem* items;
+  const int* counts;      // lists (forward lists for dQ, transposed for dK/dV)
+  const int* ids;
+  int max_k;
+  int tile_blocks;
+  int V;
+  int L_v;
+  int text_len;
+  int text_blocks;        // dQ: key blocks of the text block with valid keys
+  int text_sentinel;      // lists end with the text block
+  float scale_log2;       // log2(e) / sqrt(d)
+  float scale;            // 1 / sqrt(d)
+  const float* lse2;      // [rows] log-sum-exp in log2 units
+  const float* delta;     // [rows] D
+  __nv_bfloat16* out_a;   // dQ (dQ kernel) or dK (dK/dV kernel)
+  __nv_bfloat16* out_b;   // dV (dK/dV kernel)
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kPanelBytes = 128 * 128;
+  static constexpr int kBlockBytes = 128 * D * 2;
+  static constexpr int kStages = 2;
+  static constexpr int kResA = 0;                                  // K (dKV) / Q (dQ)
+  static constexpr int kResB = kResA + kBlockBytes;                // V (dKV) / dO (dQ)
+  static constexpr int kStream = kResB + kBlockBytes;              // per stage: 2 blocks + vec
+  static constexpr int kStageBytes = 2 * kBlockBytes + 1024;
+  static constexpr int kBarOff = kStream + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+};
+
+// One warp per two rows: D[row] = sum_c dO[row,c] * O[row,c] (fp32) and the
+// log-sum-exp converted to log2 units.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
+    const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
+    long long rows) {
+  constexpr int kLanes = D / 8;                       // 16-byte vectors per row
+  constexpr int kRowsPerWarp = 32 / kLanes;
+  const long long warp = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const long long row = warp * kRowsPerWarp + lane / kLanes;
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + lane % kLanes);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dout + row * D) + lane % kLanes);
+    const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(pa[e]);
+      const float2 fb = __bfloat1622float2(pb[e]);
+      acc = fmaf(fa.x, fb.x, acc);
+      acc = fmaf(fa.y, fb.y, acc);
+    }
+  }
+#pragma unroll
+  for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && lane % kLanes == 0) {
+    delta[row] = acc;
+    lse2[row] = lse[row] * 1.4426950408889634f;
+  }
+}
+
+// Transposed tile lists: for key tile k of window class c, the ascending query
+// tiles whose window box holds k, then the text query block NV when has_text
+// (text queries see every video key).  Row NV (text keys, when has_text):
+// every query tile, then NV.  One thread per (class, key row).
+__global__ void __launch_bounds__(128) kv_tile_list_transposed_kernel(
+    int* __restrict__ counts, int* __restrict__ ids, const ListWindows windows, int nclass,
+    ListGeom g, int has_text) {
+  const int gid = blockIdx.x * blockDim.x + threadIdx.x;
+  if (gid >= nclass * g.NQ) return;
+  const int cls = gid / g.NQ;
+  const int row = gid - cls * g.NQ;
+  int* out = ids + static_cast<size_t>(gid) * g.max_k;
+  int n = 0;
+  if (row < g.NV) {
+    const int kw = row % g.NW, kh = (row / g.NW) % g.NH, kt = row / (g.NW * g.NH);
+    for (int q = 0; q < g.NV; ++q) {
+      const int qw = q % g.NW, qh = (q / g.NW) % g.NH, qt = q / (g.NW * g.NH);
+      int s0, e0, s1, e1, s2, e2;
+      window_range(qt, windows.w[cls * 3 + 0], g.NT, s0, e0);
+      window_range(qh, windows.w[cls * 3 + 1], g.NH, s1, e1);
+      window_range(qw, windows.w[cls * 3 + 2], g.NW, s2, e2);
+      if (kt >= s0 && kt < s0 + e0 && kh >= s1 && kh < s1 + e1 && kw >= s2 && kw < s2 + e2)
+        out[n++] = q;
+    }
+  } else {
+    for (int q = 0; q < g.NV; ++q) out[n++] = q;
+  }
+  if (has_text) out[n++] = g.NV;
+  counts[gid] = n;
+  for (int i = n; i < g.max_k; ++i) out[i] = -1;
+}
+
+template <int D, bool kDKV>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                    const __grid_constant__ CUtensorMap tmap_k,
+                    const __grid_constant__ CUtensorMap tmap_v,
+                    const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int ST = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* res_full = bars;
+  uint64_t* full = res_full + 1;         // [ST]
+  uint64_t* empty = full + ST;           // [ST]
+  uint64_t* s_full = empty + ST;
+  uint64_t* p_full = s_full + 1;
+  uint64_t* acc_full = p_full + 1;
+  uint64_t* mma_done = acc_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const WorkItem item = p.items[blockIdx.x];
+  // stream: key blocks of the query block (dQ) or query blocks of the key block (dK/dV)
+  const int cnt = p.counts[item.list];
+  const int* ids = p.ids + static_cast<size_t>(item.list) * p.max_k;
+  const int nvid = (cnt - p.text_sentinel) * p.tile_blocks;
+  const int n = nvid + (p.text_sentinel ? p.text_blocks : 0);
+  auto stream_row = [&](int j) {
+    if (j < nvid) {
+      const int t = j / p.tile_blocks;
+      return item.kv_base + ids[t] * p.V + (j - t * p.tile_blocks) * 128;
+    }
+    return item.kv_base + p.L_v + (j - nvid) * 128;
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(res_full, 1);
+    for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 8);
+    mbar_init(acc_full, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+    tma_prefetch_desc(&tmap_do);
+  }
+  if (warp == 1) tmem_alloc(tmem_holder, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const bool skip = *abort_flag != 0;
+  const uint32_t s_res_a = smem_u32(smem + C::kResA);
+  const uint32_t s_res_b = smem_u32(smem + C::kResB);
+  const uint32_t s_stream = smem_u32(smem + C::kStream);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && !skip) {
+      const uint64_t pol = policy_evict_last();
+      const int row0 = item.q0;   // the resident block
+      mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
+#pragma unroll
+      for (int pn = 0; pn < C::kPanels; ++pn) {
+        tma_load_2d_hint(smem + C::kResA + pn * C::kPanelBytes, kDKV ? &tmap_k : &tmap_q,
+                         res_full, pn * 64, row0, pol);
+        tma_load_2d_hint(smem + C::kResB + pn * C::kPanelBytes, kDKV ? &tmap_v : &tmap_do,
+                         res_full, pn * 64, row0, pol);
+      }
+      int issued = 0;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % ST;
+        if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
+        const int row = stream_row(j);
+        uint8_t* base = smem + C::kStream + st * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + (kDKV ? 1024 : 0));
+#pragma unroll
+        for (int pn = 0; pn < C::kPanels; ++pn) {
+          tma_load_2d_hint(base + pn * C::kPanelBytes, kDKV ? &tmap_q : &tmap_k, &full[st],
+                           pn * 64, row, pol);
+          tma_load_2d_hint(base + C::kBlockBytes + pn * C::kPanelBytes,
+                           kDKV ? &tmap_do : &tmap_v, &full[st], pn * 64, row, pol);
+        }
+        if constexpr (kDKV) {
+          // the streamed query block's lse2 and D (2 x 512 bytes)
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+              "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes)),
+              "l"(reinterpret_cast<uint64_t>(p.lse2 + row)), "r"(smem_u32(&full[st]))
+              : "memory");
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+              "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes + 512)),
+              "l"(reinterpret_cast<uint64_t>(p.delta + row)), "r"(smem_u32(&full[st]))
+              : "memory");
+        }
+        issued = j + 1;
+      }
+      mbar_wait_drain(res_full, 0);
+      for (int s = 0; s < ST && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / ST) * ST;
+        mbar_wait_drain(&full[s], (last / ST) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !skip) {
+      constexpr uint32_t kIdS = idesc_bf16(128, 128, false);   // scores: both K-major
+      constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);    // accumulators: B MN-major
+      auto ss_mma = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
+          umma_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024),
+                  sdesc_sw128(b_smem + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
+        }
+      };
+      // acc += A (TMEM, packed bf16 in columns [a, a+32) and [a+64, a+96)) * B
+      auto ts_mma = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+          umma_ts(d_tmem, a_tmem + acol, sdesc_sw128(b_smem + kk * 16 * 128, C::kPanelBytes, 1024),
+                  kIdAcc, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(res_full, 0, abort_flag);
+      for (int j = 0; ok && j < n; ++j) {
+        const int st = j % ST;
+        if (!mbar_wait(&full[st], (j / ST) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t sa = s_stream + st * C::kStageBytes;
+        const uint32_t sb = sa + C::kBlockBytes;
+        ss_mma(tmem + 0, s_res_a, sa);      // S^T = K Q^T  |  S = Q K^T
+        ss_mma(tmem + 128, s_res_b, sb);    // dP^T = V dO^T |  dP = dO V^T
+        umma_commit(s_full);
+        if (!mbar_wait(p_full, j & 1, abort_flag)) break;
+        tc_fence_after();
+        if constexpr (kDKV) {
+          ts_mma(tmem + 256, tmem + 0, sb, j > 0);         // dV += P^T dO
+          ts_mma(tmem + 256 + D, tmem + 128, sa, j > 0);   // dK += dS^T Q
+        } else {
+          ts_mma(tmem + 256, tmem + 0, sa, j > 0);         // dQ += dS K
+        }
+        umma_commit(&empty[st]);
+        if (j == n - 1) umma_commit(acc_full);
+      }
+      umma_commit(mma_done);
+      mbar_wait_drain(mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------ elementwise
+    const int ks = warp - 2;
+    const int half = ks >> 2;
+    const int sub = warp & 3;
+    const int r = sub * 32 + lane;                      // row of the resident block
+    const int my_row = item.q0 + r;
+    if (!skip) {
+      const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
+      const uint32_t t_s = tmem + lane_off + half * 64;           // S / S^T columns
+      const uint32_t t_dp = tmem + lane_off + 128 + half * 64;    // dP / dP^T columns
+      const float sl2 = p.scale_log2;
+      // dQ: this query row's lse2 and D; dK/dV: whether this key row is valid
+      float row_lse2 = 0.f, row_delta = 0.f;
+      bool row_valid = true;
+      if constexpr (kDKV) {
+        const int off = my_row - item.kv_base;
+        if (off >= p.L_v) row_valid = (off - p.L_v) < p.text_len;
+      } else {
+        row_lse2 = p.lse2[my_row];
+        row_delta = p.delta[my_row];
+      }
+      bool done = true;
+      for (int j = 0; j < n; ++j) {
+        const int st = j % ST;
+        if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
+        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        uint32_t sr[64], dr[64];
+        STA_TMEM_LD32(t_s, (sr + 0));
+        STA_TMEM_LD32(t_s + 32, (sr + 32));
+        STA_TMEM_LD32(t_dp, (dr + 0));
+        STA_TMEM_LD32(t_dp + 32, (dr + 32));
+        tmem_wait_ld();
+        // column mask: dQ over the text key block (keys >= text_len)
+        int hi = 64;
+        if constexpr (!kDKV) {
+          if (j >= nvid) {
+            const int col0 = (j - nvid) * 128 + half * 64;
+            hi = p.text_len - col0;
+          }
+        }
+        const float* vec = reinterpret_cast<const float*>(
+            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes);
+        uint32_t pk_p[32], pk_ds[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int c = 2 * e + u;
+            const float s = __uint_as_float(sr[c]);
+            const float dp = __uint_as_float(dr[c]);
+            float lse2, dl;
+            if constexpr (kDKV) {
+              lse2 = vec[half * 64 + c];
+              dl = vec[128 + half * 64 + c];
+            } else {
+              lse2 = row_lse2;
+              dl = row_delta;
+            }
+            float pr = fast_exp2(fmaf(s, sl2, -lse2));
+            if (!row_valid || c >= hi) pr = 0.f;
+            pv[u] = pr;
+            dsv[u] = pr * (dp - dl);
+          }
+          pk_p[e] = pack_bf16x2(pv[0], pv[1]);
+          pk_ds[e] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        if constexpr (kDKV) {
+          STA_TMEM_ST32(t_s, pk_p);     // P^T over the first 32 of this warp's columns
+          STA_TMEM_ST32(t_dp, pk_ds);   // dS^T likewise in the dP^T columns
+        } else {
+          STA_TMEM_ST32(t_s, pk_ds);    // dS over the S columns
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_full);
+      }
+      if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
+        tc_fence_after();
+        constexpr int kHalfCols = D / 2;
+        const int nacc = kDKV ? 2 : 1;
+        for (int a = 0; a < nacc; ++a) {
+          // dK/dV kernel: a = 0 -> dV (unscaled), a = 1 -> dK (scaled)
+          const uint32_t t_acc = tmem + lane_off + 256 + (kDKV && a == 0 ? 0 : (kDKV ? D : 0)) +
+                                 half * kHalfCols;
+          const float sc = (kDKV && a == 0) ? 1.f : p.scale;
+          __nv_bfloat16* dstp = (kDKV && a == 0) ? p.out_b : p.out_a;
+          uint4* dst = reinterpret_cast<uint4*>(dstp + static_cast<size_t>(my_row) * D +
+                                                half * kHalfCols);
+#pragma unroll
+          for (int cc = 0; cc < kHalfCols / 32; ++cc) {
+            uint32_t o[32];
+            STA_TMEM_LD32(t_acc + cc * 32, o);
+            tmem_wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * sc, __uint_as_float(o[2 * e + 1]) * sc);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                            pk[4 * v4 + 3]);
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace sta

@@ -21,6 +21,7 @@
 #include "tile_lists.cuh"
 #include "attn_fwd.cuh"
 #include "hilbert.cuh"
+#include "attn_bwd.cuh"
 
 namespace {
 
@@ -742,6 +743,203 @@ void launch_coords_rects(uint32_t* coords, int4* rects, int n, int order, cudaSt
   sta::block_rect_kernel<<<(nb * 32 + 255) / 256, 256, 0, st>>>(coords, rects, nb);
 }
 
+// ------------------------------------------------------------------ backward
+struct BwdWs {
+  void* buf = nullptr;
+  size_t cap = 0;
+};
+BwdWs g_wsb[64];
+
+template <int D, bool kDKV>
+sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const CUtensorMap& mdo, const sta::BwdParams& prm, int num_items,
+                      cudaStream_t st) {
+  constexpr int smem = sta::BwdCfg<D>::kSmemBytes;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  STA_CUDA_TRY(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_kernel<D, kDKV>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set[dev] = true;
+  }
+  sta::attn_bwd_kernel<D, kDKV><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+  STA_CUDA_TRY(cudaGetLastError());
+  return STA_OK;
+}
+
+sta_status backward_impl(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                         int B, int heads, int d, int T, int H, int W, const int tile[3],
+                         const int* window, int text_len, int has_text, void* stream) {
+  const void* ins[6] = {q, k, v, o, dout, lse};
+  for (const void* x : ins)
+    if (!x || !aligned16(x)) return STA_ERR_INVALID_ARG;
+  const void* outs[3] = {dq, dk, dv};
+  for (const void* x : outs) {
+    if (!x || !aligned16(x)) return STA_ERR_INVALID_ARG;
+    for (const void* y : ins)
+      if (x == y) return STA_ERR_INVALID_ARG;
+  }
+  if (dq == dk || dq == dv || dk == dv || B < 1 || heads < 1) return STA_ERR_INVALID_ARG;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, text_len);
+  if (s != STA_OK) return s;
+  s = check_windows(window, heads);
+  if (s != STA_OK) return s;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  if (g.V % 128 != 0) return STA_ERR_UNSUPPORTED;
+  const int64_t rows = int64_t(B) * heads * g.S;
+  if (rows >= (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_mu);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  Classes cls = make_classes(window, heads);
+  if (cls.nclass > kMaxClasses) return STA_ERR_UNSUPPORTED;
+  const int sentinel = (g.has_text && g.text_len > 0) ? 1 : 0;
+  const int NQ = g.NV + (g.has_text ? 1 : 0);
+  const int max_k = g.NV + 1;   // both list kinds fit in NV + 1 entries
+  const int bpt = g.V / 128;
+  // workspace: lse2, delta, forward lists, transposed lists, two plans
+  const size_t vb = align_up(sizeof(float) * size_t(rows), 256);
+  const size_t cb = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
+  const size_t ib = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
+  const size_t blocks = size_t(B) * heads * (g.S / 128);
+  const size_t pb = align_up(sizeof(WorkItem) * blocks, 256);
+  const size_t total = 2 * vb + 2 * cb + 2 * ib + 2 * pb;
+  BwdWs& ws = g_wsb[dev];
+  if (ws.cap < total) {
+    if (ws.buf) STA_CUDA_TRY(cudaFree(ws.buf));
+    ws.buf = nullptr;
+    ws.cap = 0;
+    STA_CUDA_TRY(cudaMalloc(&ws.buf, total));
+    ws.cap = total;
+  }
+  uint8_t* w = static_cast<uint8_t*>(ws.buf);
+  float* lse2 = reinterpret_cast<float*>(w);
+  float* delta = reinterpret_cast<float*>(w + vb);
+  int* fc = reinterpret_cast<int*>(w + 2 * vb);
+  int* tc = reinterpret_cast<int*>(w + 2 * vb + cb);
+  int* fi = reinterpret_cast<int*>(w + 2 * vb + 2 * cb);
+  int* ti = reinterpret_cast<int*>(w + 2 * vb + 2 * cb + ib);
+  WorkItem* qitems = reinterpret_cast<WorkItem*>(w + 2 * vb + 2 * cb + 2 * ib);
+  WorkItem* kitems = reinterpret_cast<WorkItem*>(w + 2 * vb + 2 * cb + 2 * ib + pb);
+  // plans: one item per 128-row block, longest streams first
+  std::vector<std::pair<int, WorkItem>> qp, kp;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < heads; ++h) {
+      const int base = (b * heads + h) * g.S;
+      const int c = cls.head_class[h];
+      const int* wv = &cls.win[3 * c];
+      const int qlen = class_video_tiles(g, wv) * bpt + sentinel * ((g.text_len + 127) / 128);
+      for (int t = 0; t < g.NV; ++t)
+        for (int sb = 0; sb < bpt; ++sb) {
+          const int row = base + t * g.V + sb * 128;
+          qp.push_back({qlen, {row, -1, base, c * NQ + t}});
+          // key tile t is seen by the query tiles whose box holds it
+          int seen = 1;
+          for (int a = 0; a < 3; ++a) {
+            const int cc = a == 0 ? t / (g.NW * g.NH) : (a == 1 ? (t / g.NW) % g.NH : t % g.NW);
+            const int na = a == 0 ? g.NT : (a == 1 ? g.NH : g.NW);
+            int cntq = 0;
+            for (int x = 0; x < na; ++x) {
+              int s0, e0;
+              window_range_host(x, wv[a], na, &s0, &e0);
+              cntq += (cc >= s0 && cc < s0 + e0);
+            }
+            seen *= cntq;
+          }
+          kp.push_back({seen * bpt + (g.has_text ? 2 : 0), {row, -1, base, c * NQ + t}});
+        }
+      if (g.has_text) {
+        const int qtext = g.NV * bpt + sentinel * ((g.text_len + 127) / 128);
+        for (int tb = 0; tb < 2; ++tb) {
+          const int row = base + g.Lv + tb * 128;
+          qp.push_back({qtext, {row, -1, base, c * NQ + g.NV}});
+          kp.push_back({g.NV * bpt + 2, {row, -1, base, c * NQ + g.NV}});
+        }
+      }
+    }
+  auto by_len = [](const std::pair<int, WorkItem>& a, const std::pair<int, WorkItem>& b) {
+    return a.first > b.first;
+  };
+  std::stable_sort(qp.begin(), qp.end(), by_len);
+  std::stable_sort(kp.begin(), kp.end(), by_len);
+  std::vector<WorkItem> qv, kv;
+  for (auto& e : qp) qv.push_back(e.second);
+  for (auto& e : kp) kv.push_back(e.second);
+  STA_CUDA_TRY(cudaMemcpyAsync(qitems, qv.data(), sizeof(WorkItem) * qv.size(),
+                               cudaMemcpyHostToDevice, st));
+  STA_CUDA_TRY(cudaMemcpyAsync(kitems, kv.data(), sizeof(WorkItem) * kv.size(),
+                               cudaMemcpyHostToDevice, st));
+  // D and lse2
+  const long long warps = (rows * (d / 8) + 31) / 32;
+  const int pre_blocks = static_cast<int>((warps * 32 + 255) / 256);
+  if (d == 128)
+    sta::bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+        delta, lse2, rows);
+  else
+    sta::bwd_preprocess_kernel<64><<<pre_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
+        delta, lse2, rows);
+  // forward and transposed tile lists
+  launch_lists(fc, fi, cls, g, max_k, st);
+  {
+    sta::ListWindows wp;
+    std::memset(&wp, 0, sizeof(wp));
+    std::memcpy(wp.w, cls.win.data(), sizeof(int) * cls.win.size());
+    sta::ListGeom lg;
+    std::memset(&lg, 0, sizeof(lg));
+    lg.NT = g.NT; lg.NH = g.NH; lg.NW = g.NW; lg.NV = g.NV; lg.NQ = NQ; lg.max_k = max_k;
+    const int tot = cls.nclass * NQ;
+    sta::kv_tile_list_transposed_kernel<<<(tot + 127) / 128, 128, 0, st>>>(
+        tc, ti, wp, cls.nclass, lg, g.has_text ? 1 : 0);
+  }
+  STA_CUDA_TRY(cudaGetLastError());
+  CUtensorMap mq, mk, mv, mdo;
+  s = make_row_map(&mq, q, rows, d);
+  if (s == STA_OK) s = make_row_map(&mk, k, rows, d);
+  if (s == STA_OK) s = make_row_map(&mv, v, rows, d);
+  if (s == STA_OK) s = make_row_map(&mdo, dout, rows, d);
+  if (s != STA_OK) return s;
+  sta::BwdParams prm;
+  std::memset(&prm, 0, sizeof(prm));
+  prm.max_k = max_k;
+  prm.tile_blocks = bpt;
+  prm.V = g.V;
+  prm.L_v = g.Lv;
+  prm.text_len = g.text_len;
+  prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
+  prm.scale = static_cast<float>(1.0 / std::sqrt(double(d)));
+  prm.lse2 = lse2;
+  prm.delta = delta;
+  // dQ: forward lists, text key blocks with valid keys
+  prm.items = qitems;
+  prm.counts = fc;
+  prm.ids = fi;
+  prm.text_sentinel = sentinel;
+  prm.text_blocks = (g.text_len + 127) / 128;
+  prm.out_a = static_cast<__nv_bfloat16*>(dq);
+  prm.out_b = nullptr;
+  s = d == 128 ? launch_bwd<128, false>(mq, mk, mv, mdo, prm, int(qv.size()), st)
+               : launch_bwd<64, false>(mq, mk, mv, mdo, prm, int(qv.size()), st);
+  if (s != STA_OK) return s;
+  // dK, dV: transposed lists, the 256 text query rows as two blocks
+  prm.items = kitems;
+  prm.counts = tc;
+  prm.ids = ti;
+  prm.text_sentinel = g.has_text ? 1 : 0;
+  prm.text_blocks = 2;
+  prm.out_a = static_cast<__nv_bfloat16*>(dk);
+  prm.out_b = static_cast<__nv_bfloat16*>(dv);
+  return d == 128 ? launch_bwd<128, true>(mq, mk, mv, mdo, prm, int(kv.size()), st)
+                  : launch_bwd<64, true>(mq, mk, mv, mdo, prm, int(kv.size()), st);
+}
+
 }  // namespace
 
 // ====================================================================== C ABI
@@ -1029,6 +1227,14 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void
   return launch_attn<64, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
 }
 
+sta_status sta_backward(const void* q, const void* k, const void* v, const void* out,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int B, int heads, int d, int T, int H, int W, const int tile[3],
+                        const int* window, int text_len, int has_text, void* stream) {
+  return backward_impl(q, k, v, out, dout, lse, dq, dk, dv, B, heads, d, T, H, W, tile, window,
+                       text_len, has_text, stream);
+}
+
 sta_status sta_device_status(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return STA_ERR_CUDA;
@@ -1052,6 +1258,11 @@ void sta_shutdown(void) {
       cudaSetDevice(i);
       cudaFree(g_ws[i].buf);
       g_ws[i] = Workspace();
+    }
+    if (g_wsb[i].buf != nullptr) {
+      cudaSetDevice(i);
+      cudaFree(g_wsb[i].buf);
+      g_wsb[i] = BwdWs();
     }
     if (g_ws2d[i].buf != nullptr) {
       cudaSetDevice(i);

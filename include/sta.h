@@ -129,6 +129,25 @@ sta_status sta_forward_raster(const void* q, const void* k, const void* v,
                               void* stream);
 
 /*
+ * sta_backward - gradients of sta_forward (STA backward pass; the pages give
+ * the forward only, the backward is its gradient).  All tensors TILE order,
+ * [B, heads, S, d] bf16 device: q, k, v, out (the forward output), dout
+ * (gradient of the loss w.r.t. out); lse: device fp32 [B, heads, S] from
+ * sta_forward_lse.  Writes dq, dk, dv (bf16, same layout; caller-owned,
+ * distinct from the inputs).  With P = softmax(q k^T / sqrt(d)) on allowed
+ * pairs and D = rowsum(dout * out): dv = P^T dout, dS = P (dout v^T - D),
+ * dq = dS k / sqrt(d), dk = dS^T q / sqrt(d); padded text keys get zero.
+ * fp32 accumulation in tensor memory, P and dS rounded to bf16 for the MMAs.
+ * Same geometry limits as sta_forward.
+ */
+sta_status sta_backward(const void* q, const void* k, const void* v,
+                        const void* out, const void* dout, const float* lse,
+                        void* dq, void* dk, void* dv, int B, int heads, int d,
+                        int T, int H, int W, const int tile[3],
+                        const int* window, int text_len, int has_text,
+                        void* stream);
+
+/*
  * sta_swa_forward - token-level sliding-window attention with grouped-query
  * heads, the mixed-block baseline of README "Why is STA Fast?"; the 1-D
  * causal window over the previous `window` positions (self included) with
