@@ -34,8 +34,6 @@
 // reads P_i; tcgen05 MMAs of one thread execute in issue order.
 #pragma once
 
-#include <type_traits>
-
 #include "device_ptx.cuh"
 
 namespace sta {
@@ -192,16 +190,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
       return false;
     }
   }
-}
-
-// Pairs of score columns (of the 16 pairs of each 32-column group) whose
-// exp2 is evaluated by exp2_poly on the FMA pipe instead of MUFU, spread
-// evenly; unmasked blocks only.
-#ifndef STA_EXP2_POLY_PAIRS
-#define STA_EXP2_POLY_PAIRS 0
-#endif
-__device__ __forceinline__ constexpr bool kPolyPair(int e) {
-  return (e * STA_EXP2_POLY_PAIRS) % 16 >= 16 - STA_EXP2_POLY_PAIRS;
 }
 
 // Loads one 128-row block whose first row in the tile-ordered view is `row`
@@ -535,8 +523,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
         for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
         int lo, hi;
-        bool masked = seq_mask<M>(p, seq, j, r, lo, hi);
-        if (masked) {
+        if (seq_mask<M>(p, seq, j, r, lo, hi)) {
           lo -= half * kCols;
           hi -= half * kCols;
 #pragma unroll
@@ -559,7 +546,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 s[c4 * 4 + e] = -INFINITY;
             }
           }
-          masked = true;
         }
         if constexpr (M == Mode::kSwa3d) {
           static_assert(kSplit == 2, "the 3-D window mask gives each half one t-slice");
@@ -574,7 +560,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
             for (int c = 0; c < kCols; ++c)
               if (!((km >> c) & 1ull)) s[c] = -INFINITY;
-            masked = true;
           }
         }
         float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
@@ -602,32 +587,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           l_run *= alpha;
         }
         const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        // exp2 of the scaled, shifted scores -> bf16 P in TMEM
         float ls0 = 0.f, ls1 = 0.f;
-        // exp2 of the scaled, shifted scores -> bf16 P in TMEM; on unmasked
-        // blocks a share of the pairs goes to the FMA-pipe polynomial.
-        auto exp_block = [&](auto use_poly) {
-          constexpr bool kPoly = decltype(use_poly)::value;
 #pragma unroll
-          for (int cc = 0; cc < kCols / 32; ++cc) {
-            uint32_t pk[16];
+        for (int cc = 0; cc < kCols / 32; ++cc) {
+          uint32_t pk[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float x0 = fmaf(s[cc * 32 + 2 * e], sl2, neg_m);
-              const float x1 = fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m);
-              const bool poly = kPoly && kPolyPair(e);
-              const float p0 = poly ? exp2_poly(x0) : fast_exp2(x0);
-              const float p1 = poly ? exp2_poly(x1) : fast_exp2(x1);
-              ls0 += p0;
-              ls1 += p1;
-              pk[e] = pack_bf16x2(p0, p1);
-            }
-            STA_TMEM_ST16(t_p + cc * 16, pk);
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
+            const float p1 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
+            ls0 += p0;
+            ls1 += p1;
+            pk[e] = pack_bf16x2(p0, p1);
           }
-        };
-        if (masked) {
-          exp_block(std::false_type{});
-        } else {
-          exp_block(std::true_type{});
+          STA_TMEM_ST16(t_p + cc * 16, pk);
         }
         l_run += ls0 + ls1;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {

@@ -302,22 +302,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// 2^x on the FMA pipe (no MUFU): x = j + f with j = round(x) added to the
-// exponent field and 2^f, f in [-1/2, 1/2], from a degree-3 polynomial that
-// minimises the largest relative error on that interval (7.5e-5; fitted by
-// block_sparse_local_b200/exp2_poly.py, Cody & Waite style range reduction).
-// Arguments below -125 are clamped, so the result is a normal float; use it
-// only where every argument is finite.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -125.f);
-  const float t = x + 12582912.f;          // 1.5 * 2^23: low bits hold round(x)
-  const float f = x - (t - 12582912.f);
-  float p = fmaf(0.0551722199f, f, 0.242611155f);
-  p = fmaf(p, f, 0.693260849f);
-  p = fmaf(p, f, 0.999928057f);
-  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
-}
-
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
