@@ -125,6 +125,7 @@ RASTER_CASES = [
     ((1, 64, 64), (1, 16, 16), [(1, 3, 3)], 0, False, 64, 2),               # box 16x8x1
     ((4, 24, 32), (2, 8, 8), [(1, 3, 3), (2, 2, 4)], 37, True, 128, 1),      # 128-token tiles
     ((8, 32, 16), (2, 16, 8), [(3, 1, 2)], 129, True, 64, 1),               # box 8x16x1
+    ((12, 16, 24), (6, 8, 8), [(1, 2, 3), (3, 1, 1), (1, 2, 3)], 5, True, 64, 2),  # B=2
 ]
 
 

@@ -43,6 +43,7 @@ CASES = [
     ((4, 16, 24), (2, 8, 8), [(2, 1, 3), (1, 2, 1)], 77, True, 128),
     ((6, 8, 16), (6, 8, 8), [(1, 1, 2)], 200, True, 64),
     ((4, 8, 16), (2, 8, 8), [(2, 1, 2)], 256, True, 128),
+    ((4, 8, 16), (2, 8, 8), [(1, 1, 1)], 0, True, 64),    # text rows, no valid text key
 ]
 
 

@@ -46,7 +46,7 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
     first = workloads.small_sta_case(base.T, base.H, base.W, base.tile, [(3, 3, 3)] * 3,
                                      base.text_len, True, d=128, seed=21)
     second = workloads.small_sta_case(12, 16, 24, (6, 8, 8), [(1, 2, 3), (2, 2, 2)], 77, True,
-                                      d=64, B=2, seed=22)
+                                      d=64, B=2, seed=22)   # two window classes, text
     for w in (first, second):
         q, k, v = workloads.sta_inputs(w, device="cuda")
         shape = (w.T, w.H, w.W)
