@@ -39,10 +39,21 @@ ATTN_SOURCES = ("block_sparse_local_b200/csrc/attn_fwd.cuh",
                 "block_sparse_local_b200/csrc/device_ptx.cuh")
 
 
+def workload_config(w, world):
+    """The `config` object of the JSON line (both arms)."""
+    return {"workload": w.name, "B_per_gpu": w.B, "heads": w.heads, "d": w.d,
+            "video": [w.T, w.H, w.W], "tile": list(w.tile), "window": list(w.windows[0]),
+            "text_len": w.text_len, "seq_len": w.S, "global_batch": w.B * world,
+            "parallelism": f"independent problems x{world}",
+            "l2": "inputs larger than L2 (3 x 710 MB), no flush",
+            "step": "tile lists + attention with the raster<->tile permutation "
+                    "fused into its TMA loads and output stores"}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -103,7 +114,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
@@ -206,9 +217,8 @@ def run_reference(args):
         "ms_per_step": flops / (value * 1e12) * 1e3 if value > 0 else None,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "d": w.d,
-                   "video": [w.T, w.H, w.W], "tile": list(w.tile), "window": list(w.windows[0]),
-                   "text_len": w.text_len, "seq_len": w.S, "note": "ms_per_step extrapolated"},
+        "config": workload_config(w, args.gpus),
+        "note": "CPU oracle on a bounded sample; ms_per_step extrapolated to the whole workload",
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -476,14 +486,7 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "B_per_gpu": w.B, "heads": w.heads, "d": w.d,
-                       "video": [w.T, w.H, w.W], "tile": list(w.tile),
-                       "window": list(w.windows[0]), "text_len": w.text_len,
-                       "seq_len": w.S, "global_batch": w.B * world,
-                       "parallelism": f"independent problems x{world}",
-                       "l2": "inputs larger than L2 (3 x 710 MB), no flush",
-                       "step": "tile lists + attention with the raster<->tile permutation "
-                               "fused into its TMA loads and output stores"},
+            "config": workload_config(w, world),
             "pct_of_bf16_peak": 100.0 * value / peak,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 2 * args.steps, "permutation": perm, "swa_comparison": swa,

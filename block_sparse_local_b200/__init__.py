@@ -22,7 +22,7 @@ __all__ = [
     "forward", "sliding_tile_attention", "swa_forward", "device_status",
     "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
     "hilbert_reorder", "build_slide_block_lists", "slide2d_forward", "slide_attention_2d",
-    "backward", "SlidingTileAttentionFunction",
+    "backward", "SlidingTileAttentionFunction", "TileReorderFunction",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -248,6 +248,22 @@ class SlidingTileAttentionFunction(torch.autograd.Function):
         return dq, dk, dv, None, None, None, None, None
 
 
+class TileReorderFunction(torch.autograd.Function):
+    """Differentiable raster -> tile permutation (its gradient is the inverse)."""
+
+    @staticmethod
+    def forward(ctx, x, video_shape, tile, has_text, to_tile):
+        ctx.args = (video_shape, tile, has_text, to_tile)
+        f = tile_reorder if to_tile else tile_unreorder
+        return f(x.contiguous(), video_shape, tile, has_text)
+
+    @staticmethod
+    def backward(ctx, g):
+        video_shape, tile, has_text, to_tile = ctx.args
+        f = tile_unreorder if to_tile else tile_reorder
+        return f(g.contiguous(), video_shape, tile, has_text), None, None, None, None
+
+
 def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
                            video_shape=(30, 48, 80), tile=(6, 8, 8), fused=True):
     """README-style call on RASTER-ordered q, k, v.
@@ -255,7 +271,16 @@ def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
     fused=True: one attention kernel reads and writes raster order directly
     (sta_forward_raster); tile shapes whose blocks are not boxes of the grid
     go through the explicit reorder -> attend -> unreorder kernels instead.
+    When an input requires grad, the call is differentiable (permutation,
+    attention with saved log-sum-exp, inverse permutation; backward by
+    sta_backward).
     """
+    if torch.is_grad_enabled() and any(t.requires_grad for t in (q, k, v)):
+        qt, kt, vt = (TileReorderFunction.apply(x, video_shape, tile, has_text, True)
+                      for x in (q, k, v))
+        ot = SlidingTileAttentionFunction.apply(qt, kt, vt, window_size, text_length,
+                                                has_text, video_shape, tile)
+        return TileReorderFunction.apply(ot, video_shape, tile, has_text, False)
     if fused:
         try:
             return forward_raster(q, k, v, window_size, text_length, has_text, video_shape,

@@ -109,3 +109,23 @@ def test_backward_full_size_dq_sampled():
         _close(dq[0, h].float().cpu().numpy()[rows], ref, f"dq h{h}")
     for x in (dk, dv):
         assert torch.isfinite(x.float()).all()
+
+
+def test_raster_api_is_differentiable():
+    w = workloads.small_sta_case(4, 16, 24, (2, 8, 8), [(1, 2, 2), (2, 1, 3)], 33, True, d=128,
+                                 seed=47)
+    q, k, v = workloads.sta_inputs(w)
+    dout = workloads.randn_bf16(q.shape, 4747)
+    qd, kd, vd = (x.cuda().requires_grad_() for x in (q, k, v))
+    out = sta.sliding_tile_attention(qd, kd, vd, w.windows, w.text_len, True, (w.T, w.H, w.W),
+                                     w.tile)
+    out.backward(dout.cuda())
+    sta.device_status()
+    for h in range(w.heads):
+        x64 = [x[0, h].double().numpy() for x in (q, k, v, dout)]
+        rdq, rdk, rdv, rout, _ = sta_bwd_oracle.sta_backward_dense(
+            *x64, w.T, w.H, w.W, w.tile, w.windows[h], w.text_len, True)
+        _close(out[0, h].detach().float().cpu().numpy(), rout, f"out h{h}")
+        _close(qd.grad[0, h].float().cpu().numpy(), rdq, f"dq h{h}")
+        _close(kd.grad[0, h].float().cpu().numpy(), rdk, f"dk h{h}")
+        _close(vd.grad[0, h].float().cpu().numpy(), rdv, f"dv h{h}")
