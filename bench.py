@@ -309,10 +309,11 @@ def run_ours(args):
         hout = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
 
         def e2e_step():
-            dq, dk, dv = (x.to(dev, non_blocking=True) for x in (hq, hk, hv))
-            o = sta.sliding_tile_attention(dq, dk, dv, w.windows, w.text_len, w.has_text,
-                                           shape, w.tile)
-            hout.copy_(o, non_blocking=True)
+            # the README call on host tensors: the library streams chunks of
+            # heads through device staging buffers, copies overlapping compute
+            sta.sliding_tile_attention_host(hq, hk, hv, w.windows, w.text_len, w.has_text,
+                                            shape, w.tile, out=hout, device=dev,
+                                            blocking=False)
 
         for _ in range(2):
             e2e_step()

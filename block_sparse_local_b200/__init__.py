@@ -23,6 +23,7 @@ __all__ = [
     "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
     "hilbert_reorder", "build_slide_block_lists", "slide2d_forward", "slide_attention_2d",
     "backward", "SlidingTileAttentionFunction", "TileReorderFunction",
+    "sliding_tile_attention_host",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -33,7 +34,8 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_device_status", "sta_status_string", "sta_shutdown",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
             "sta_swa3d_forward", "sta_debug_inject", "sta_hilbert_reorder",
-            "sta_build_slide_block_lists", "sta_slide2d_forward", "sta_backward")
+            "sta_build_slide_block_lists", "sta_slide2d_forward", "sta_backward",
+            "sta_forward_raster_host")
 
 
 class StaError(RuntimeError):
@@ -71,6 +73,7 @@ def lib():
     L.sta_forward_noalloc.argtypes = [_P, _P, _P, _P] + fwd
     L.sta_forward_raster.argtypes = [_P, _P, _P, _P, _P] + fwd
     L.sta_swa3d_forward.argtypes = [_P, _P, _P, _P] + fwd
+    L.sta_forward_raster_host.argtypes = [_P, _P, _P, _P] + fwd[:-1] + [ctypes.c_size_t, _P]
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_debug_inject.argtypes = [_I, _I]
@@ -293,6 +296,47 @@ def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
     vt = tile_reorder(v, video_shape, tile, has_text)
     ot = forward(qt, kt, vt, window_size, text_length, has_text, video_shape, tile)
     return tile_unreorder(ot, video_shape, tile, has_text)
+
+
+def sliding_tile_attention_host(q, k, v, window_size, text_length, has_text=True,
+                                video_shape=(30, 48, 80), tile=(6, 8, 8), out=None,
+                                device=None, blocking=True, chunk_bytes=0):
+    """The README call on HOST tensors (sta_forward_raster_host).
+
+    q, k, v: CPU bf16 [B, heads, S, d], raster order, contiguous; pin them
+    (``tensor.pin_memory()``) so the copies overlap the attention.  The
+    library streams whole heads through device staging buffers on
+    ``device`` (default: the current CUDA device), at most ``chunk_bytes``
+    per tensor and chunk (0: the library default), and writes ``out``, a CPU
+    tensor (pinned when allocated here).  With blocking=False the call only
+    enqueues the work on the device's current stream: synchronise that stream
+    before reading ``out`` or touching q, k, v.
+    """
+    for t in (q, k, v):
+        if t.is_cuda or t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("tensors must be contiguous bf16 CPU tensors")
+    if not (q.shape == k.shape == v.shape):
+        raise ValueError("q, k, v must have one shape")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+    if out is None:
+        out = torch.empty(q.shape, dtype=q.dtype, pin_memory=True)
+    elif out.is_cuda or out.shape != q.shape or out.dtype != q.dtype or \
+            not out.is_contiguous():
+        raise ValueError("out must be a contiguous bf16 CPU tensor shaped like q")
+    B, nh, S, d = q.shape
+    T, H, W = video_shape
+    with torch.cuda.device(dev):
+        stream = torch.cuda.current_stream(dev)
+        _check(lib().sta_forward_raster_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), B, nh, d,
+                                             T, H, W, _I3(*tile), _windows(window_size, nh),
+                                             int(text_length), int(has_text),
+                                             int(chunk_bytes),
+                                             ctypes.c_void_p(stream.cuda_stream)),
+               "sta_forward_raster_host")
+        if blocking:
+            stream.synchronize()
+    return out
 
 
 def swa3d_forward(q, k, v, window_tokens, text_length, has_text, video_shape,

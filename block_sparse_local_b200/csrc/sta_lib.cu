@@ -158,6 +158,13 @@ void window_range_host(int c, int w, int n, int* s, int* e) {
   if (*s > n - *e) *s = n - *e;
 }
 
+// Raster-order kernels load every 128-row block of a tile as one box
+// {cw, bh, bt} of whole tile rows: cw | 128 and (ch*cw | 128 or 128 | ch*cw).
+bool raster_boxes_ok(const Geom& g) {
+  const int plane = g.ch * g.cw;
+  return 128 % g.cw == 0 && (128 % plane == 0 || plane % 128 == 0);
+}
+
 sta_status check_windows(const int* window, int heads) {
   if (window == nullptr) return STA_ERR_INVALID_ARG;
   for (int h = 0; h < heads; ++h)
@@ -409,8 +416,7 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   // whole rows of the tile (cw | 128, and ch*cw | 128 or 128 | ch*cw).
   int box_h = 0, box_t = 0;
   if (raster) {
-    const int plane = g.ch * g.cw;
-    if (128 % g.cw != 0 || !(128 % plane == 0 || plane % 128 == 0)) return STA_ERR_UNSUPPORTED;
+    if (!raster_boxes_ok(g)) return STA_ERR_UNSUPPORTED;
     box_h = std::min(g.ch, 128 / g.cw);
     box_t = 128 / (g.cw * box_h);
     if (B * int64_t(heads) > (int64_t(1) << 31)) return STA_ERR_INVALID_ARG;
@@ -515,6 +521,128 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (token_mode) return STA_ERR_UNSUPPORTED;
   if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
   return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+}
+
+// ------------------------------------------------------------------ host-buffer pipeline
+// sta_forward_raster_host: q, k, v and out live in host memory.  The (batch,
+// head) slices are independent problems, so the call walks them in chunks of
+// whole heads through two device staging buffers: the copy-in of chunk c+1
+// (stream s_in), the attention of chunk c (the caller's stream) and the
+// copy-out of chunk c-1 (stream s_out) run at the same time.
+struct HostPipe {
+  bool ready = false;
+  bool used = false;
+  cudaStream_t s_in = nullptr, s_out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_ready[2] = {}, comp_done[2] = {}, out_done[2] = {};
+  void* buf = nullptr;   // [2 buffers][q, k, v, out][chunk bytes]
+  size_t cap = 0;
+};
+HostPipe g_pipe[64];
+std::mutex g_pipe_mu;
+
+sta_status host_pipe_setup(HostPipe& hp, size_t bytes) {
+  if (!hp.ready) {
+    STA_CUDA_TRY(cudaStreamCreateWithFlags(&hp.s_in, cudaStreamNonBlocking));
+    STA_CUDA_TRY(cudaStreamCreateWithFlags(&hp.s_out, cudaStreamNonBlocking));
+    cudaEvent_t* evs[] = {&hp.start, &hp.end, &hp.in_ready[0], &hp.in_ready[1],
+                          &hp.comp_done[0], &hp.comp_done[1], &hp.out_done[0],
+                          &hp.out_done[1]};
+    for (cudaEvent_t* e : evs) STA_CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+    hp.ready = true;
+  }
+  if (hp.cap < bytes) {
+    if (hp.buf != nullptr) {
+      // the previous call's copies may still read or write the old buffer
+      STA_CUDA_TRY(cudaEventSynchronize(hp.end));
+      STA_CUDA_TRY(cudaFree(hp.buf));
+      hp.buf = nullptr;
+      hp.cap = 0;
+    }
+    STA_CUDA_TRY(cudaMalloc(&hp.buf, bytes));
+    hp.cap = bytes;
+  }
+  return STA_OK;
+}
+
+sta_status forward_host_impl(const void* q, const void* k, const void* v, void* out, int B,
+                             int heads, int d, int T, int H, int W, const int tile[3],
+                             const int* window, int text_len, int has_text,
+                             size_t chunk_bytes_max, void* stream) {
+  if (!q || !k || !v || !out) return STA_ERR_INVALID_ARG;
+  if (B < 1 || heads < 1) return STA_ERR_INVALID_ARG;
+  if (out == q || out == k || out == v) return STA_ERR_INVALID_ARG;
+  if (chunk_bytes_max == 0) chunk_bytes_max = STA_HOST_CHUNK_BYTES;
+  Geom g;
+  sta_status s = make_geom(&g, T, H, W, tile, has_text, text_len);
+  if (s != STA_OK) return s;
+  s = check_windows(window, heads);
+  if (s != STA_OK) return s;
+  if (d != 64 && d != 128) return STA_ERR_UNSUPPORTED;
+  if (g.V % sta::kBM != 0 || !raster_boxes_ok(g)) return STA_ERR_UNSUPPORTED;
+  if (make_classes(window, heads).nclass > kMaxClasses) return STA_ERR_UNSUPPORTED;
+  int dev = 0;
+  s = current_device(&dev);
+  if (s != STA_OK) return s;
+  if (!g_dev[dev].sm100) return STA_ERR_UNSUPPORTED;
+
+  const size_t slice_bytes = size_t(g.S) * d * sizeof(__nv_bfloat16);
+  const int hc = static_cast<int>(std::max<size_t>(
+      1, std::min<size_t>(size_t(heads), chunk_bytes_max / slice_bytes)));
+  const size_t chunk_bytes = size_t(hc) * slice_bytes;
+
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe& hp = g_pipe[dev];
+  s = host_pipe_setup(hp, 8 * chunk_bytes);
+  if (s != STA_OK) return s;
+  uint8_t* base = static_cast<uint8_t*>(hp.buf);
+  auto staged = [&](int buf, int tensor) { return base + (buf * 4 + tensor) * chunk_bytes; };
+  const uint8_t* src[3] = {static_cast<const uint8_t*>(q), static_cast<const uint8_t*>(k),
+                           static_cast<const uint8_t*>(v)};
+  uint8_t* dst = static_cast<uint8_t*>(out);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  // Everything earlier on the caller's stream, and every copy of the previous
+  // call (which may have come on another stream), precedes this call.
+  STA_CUDA_TRY(cudaEventRecord(hp.start, st));
+  STA_CUDA_TRY(cudaStreamWaitEvent(hp.s_in, hp.start, 0));
+  STA_CUDA_TRY(cudaStreamWaitEvent(hp.s_out, hp.start, 0));
+  if (hp.used) {
+    STA_CUDA_TRY(cudaStreamWaitEvent(hp.s_in, hp.end, 0));
+    STA_CUDA_TRY(cudaStreamWaitEvent(st, hp.end, 0));
+  }
+  hp.used = true;
+  int c = 0;
+  for (int b = 0; b < B; ++b) {
+    for (int h0 = 0; h0 < heads; h0 += hc, ++c) {
+      const int n = std::min(hc, heads - h0);
+      const int buf = c & 1;
+      const size_t off = (size_t(b) * heads + h0) * slice_bytes;
+      const size_t bytes = size_t(n) * slice_bytes;
+      // inputs of buffer `buf` are free once chunk c-2's attention has run
+      if (c >= 2) STA_CUDA_TRY(cudaStreamWaitEvent(hp.s_in, hp.comp_done[buf], 0));
+      for (int t = 0; t < 3; ++t)
+        STA_CUDA_TRY(cudaMemcpyAsync(staged(buf, t), src[t] + off, bytes,
+                                     cudaMemcpyHostToDevice, hp.s_in));
+      STA_CUDA_TRY(cudaEventRecord(hp.in_ready[buf], hp.s_in));
+      STA_CUDA_TRY(cudaStreamWaitEvent(st, hp.in_ready[buf], 0));
+      // its output is free once chunk c-2 has been copied out
+      if (c >= 2) STA_CUDA_TRY(cudaStreamWaitEvent(st, hp.out_done[buf], 0));
+      s = forward_impl(staged(buf, 0), staged(buf, 1), staged(buf, 2), staged(buf, 3),
+                       nullptr, 1, n, d, T, H, W, tile, window + 3 * h0, text_len, has_text,
+                       st, true);
+      if (s != STA_OK) return s;
+      STA_CUDA_TRY(cudaEventRecord(hp.comp_done[buf], st));
+      STA_CUDA_TRY(cudaStreamWaitEvent(hp.s_out, hp.comp_done[buf], 0));
+      STA_CUDA_TRY(cudaMemcpyAsync(dst + off, staged(buf, 3), bytes, cudaMemcpyDeviceToHost,
+                                   hp.s_out));
+      STA_CUDA_TRY(cudaEventRecord(hp.out_done[buf], hp.s_out));
+    }
+  }
+  // the caller's stream completes only after the last byte of out is home
+  STA_CUDA_TRY(cudaEventRecord(hp.end, hp.s_out));
+  STA_CUDA_TRY(cudaStreamWaitEvent(st, hp.end, 0));
+  return STA_OK;
 }
 
 template <int kVec>
@@ -1235,6 +1363,14 @@ sta_status sta_backward(const void* q, const void* k, const void* v, const void*
                        text_len, has_text, stream);
 }
 
+sta_status sta_forward_raster_host(const void* q, const void* k, const void* v, void* out,
+                                   int B, int heads, int d, int T, int H, int W,
+                                   const int tile[3], const int* window, int text_len,
+                                   int has_text, size_t chunk_bytes, void* stream) {
+  return forward_host_impl(q, k, v, out, B, heads, d, T, H, W, tile, window, text_len,
+                           has_text, chunk_bytes, stream);
+}
+
 sta_status sta_device_status(void* stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(st) != cudaSuccess) return STA_ERR_CUDA;
@@ -1268,6 +1404,22 @@ void sta_shutdown(void) {
       cudaSetDevice(i);
       cudaFree(g_ws2d[i].buf);
       g_ws2d[i] = Slide2dWs();
+    }
+  }
+  {
+    std::lock_guard<std::mutex> plock(g_pipe_mu);
+    for (int i = 0; i < 64; ++i) {
+      HostPipe& hp = g_pipe[i];
+      if (!hp.ready) continue;
+      cudaSetDevice(i);
+      cudaEventSynchronize(hp.end);
+      if (hp.buf != nullptr) cudaFree(hp.buf);
+      cudaStreamDestroy(hp.s_in);
+      cudaStreamDestroy(hp.s_out);
+      cudaEvent_t evs[] = {hp.start, hp.end, hp.in_ready[0], hp.in_ready[1], hp.comp_done[0],
+                           hp.comp_done[1], hp.out_done[0], hp.out_done[1]};
+      for (cudaEvent_t e : evs) cudaEventDestroy(e);
+      hp = HostPipe();
     }
   }
   cudaSetDevice(dev);

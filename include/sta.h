@@ -32,6 +32,7 @@
 #ifndef STA_H_
 #define STA_H_
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -127,6 +128,37 @@ sta_status sta_forward_raster(const void* q, const void* k, const void* v,
                               int T, int H, int W, const int tile[3],
                               const int* window, int text_len, int has_text,
                               void* stream);
+
+/* Default staging chunk of sta_forward_raster_host: whole heads of up to
+ * this many bytes per tensor (at least one head). */
+#define STA_HOST_CHUNK_BYTES (64u << 20)
+
+/*
+ * sta_forward_raster_host - sta_forward_raster on HOST buffers (same
+ * README Usage call, same arguments, layout and numerics; no lse).
+ * q, k, v, out: host bf16 [B, heads, S, d], raster order; page-locked
+ * (cudaHostAlloc / cudaHostRegister) for the copies to overlap, pageable
+ * memory works but serialises.  The (batch, head) slices are independent, so
+ * the call moves them in chunks of whole heads (at most `chunk_bytes` per
+ * tensor, at least one head; 0 = STA_HOST_CHUNK_BYTES) through two
+ * library-owned device staging buffers: copy-in of the
+ * next chunk, attention of the current one and copy-out of the previous one
+ * overlap on two internal streams and `stream`.  Asynchronous: `out` is
+ * complete once `stream` has reached this point (e.g. after
+ * cudaStreamSynchronize(stream)); q, k, v must stay unchanged until then.
+ * The staging buffers (8 chunks, 2 x {q,k,v,out}) grow on demand and are
+ * released by sta_shutdown(); calls on one device are serialised by the
+ * library (a later call waits, on the GPU, for the earlier one's copies).
+ * Errors: as sta_forward_raster; checked before anything is enqueued, except
+ * STA_ERR_CUDA from a failing copy or launch, which may leave `out` partly
+ * written.
+ */
+sta_status sta_forward_raster_host(const void* q, const void* k, const void* v,
+                                   void* out, int B, int heads, int d, int T,
+                                   int H, int W, const int tile[3],
+                                   const int* window, int text_len,
+                                   int has_text, size_t chunk_bytes,
+                                   void* stream);
 
 /*
  * sta_backward - gradients of sta_forward (STA backward pass; the pages give

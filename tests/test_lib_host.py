@@ -106,6 +106,21 @@ def test_reorder_and_lists_reject_bad_args(L):
                                      _wins((1, 3, -1)), 0, 0, None) == 1
 
 
+def test_host_forward_rejects_bad_args(L):
+    geo = (18, 24, 32, _i3(6, 8, 8))
+    f = L.sta_forward_raster_host
+    assert f(None, FAKE2, FAKE3, FAKE4, 1, 1, 64, *geo, _wins((1, 3, 3)), 0, 0, 0, None) == 1
+    assert f(FAKE, FAKE2, FAKE3, FAKE, 1, 1, 64, *geo, _wins((1, 3, 3)), 0, 0, 0, None) == 1
+    assert f(FAKE, FAKE2, FAKE3, FAKE4, 1, 0, 64, *geo, _wins((1, 3, 3)), 0, 0, 0, None) == 1
+    assert f(FAKE, FAKE2, FAKE3, FAKE4, 1, 1, 64, *geo, _wins((1, 0, 3)), 0, 0, 0, None) == 1
+    assert f(FAKE, FAKE2, FAKE3, FAKE4, 1, 1, 64, 18, 24, 30, _i3(6, 8, 8),
+             _wins((1, 3, 3)), 0, 0, 0, None) == 1
+    assert f(FAKE, FAKE2, FAKE3, FAKE4, 1, 1, 96, *geo, _wins((1, 3, 3)), 0, 0, 0, None) == 2
+    # (4, 2, 48) tiles (384 tokens): a 128-row block is not a box of the grid
+    assert f(FAKE, FAKE2, FAKE3, FAKE4, 1, 1, 64, 4, 2, 48, _i3(4, 2, 48),
+             _wins((1, 1, 1)), 0, 0, 0, None) == 2
+
+
 def test_swa_rejects_bad_args(L):
     assert L.sta_swa_forward(FAKE, FAKE2, FAKE3, FAKE4, 1, 6, 4, 128, 1024, 64, 1, None) == 1
     assert L.sta_swa_forward(FAKE, FAKE2, FAKE3, FAKE4, 1, 8, 4, 128, 1000, 64, 1, None) == 2
