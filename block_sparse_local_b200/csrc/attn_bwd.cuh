@@ -128,6 +128,31 @@ __global__ void __launch_bounds__(128) kv_tile_list_transposed_kernel(
   for (int i = n; i < g.max_k; ++i) out[i] = -1;
 }
 
+// D = A B^T over d (SS, both K-major, 128 x 128 scores).  a, b: descriptors
+// of the two 128-row blocks (address field already offset).
+template <int D>
+__device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint64_t a, uint64_t b) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+    umma_ss(d_tmem, a + off, b + off, kIdS, kk > 0 ? 1u : 0u);
+  }
+}
+
+// acc (+)= A B with A packed bf16 in TMEM columns [a, a+32) and [a+64, a+96)
+// (K = 128 rows of the streamed block) and B an MN-major block (N = d).
+template <int D, bool ACC>
+__device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
+  constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+    umma_ts(d_tmem, a_tmem + acol, b + ((kk * 16 * 128) >> 4), kIdAcc, (ACC || kk > 0) ? 1u : 0u);
+  }
+}
+
 template <int D, bool kDKV>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -242,48 +267,52 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !skip) {
-      constexpr uint32_t kIdS = idesc_bf16(128, 128, false);   // scores: both K-major
-      constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);    // accumulators: B MN-major
-      auto ss_mma = [&](uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024),
-                  sdesc_sw128(b_smem + off, 16, 1024), kIdS, kk > 0 ? 1u : 0u);
-        }
-      };
-      // acc += A (TMEM, packed bf16 in columns [a, a+32) and [a+64, a+96)) * B
-      auto ts_mma = [&](uint32_t d_tmem, uint32_t a_tmem, uint32_t b_smem, bool acc) {
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
-          umma_ts(d_tmem, a_tmem + acol, sdesc_sw128(b_smem + kk * 16 * 128, C::kPanelBytes, 1024),
-                  kIdAcc, (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(res_full, 0, abort_flag);
+    // Whole warp waits, one elected lane (always the same) issues; every MMA
+    // operand is warp-uniform and every accumulate flag a constant.
+    if (!skip) {
+      const uint32_t tm = warp_uniform(tmem);
+      const uint64_t d_res_a = sdesc_sw128(warp_uniform(s_res_a), 16, 1024);
+      const uint64_t d_res_b = sdesc_sw128(warp_uniform(s_res_b), 16, 1024);
+      const uint64_t d_str_k = sdesc_sw128(warp_uniform(s_stream), 16, 1024);
+      const uint64_t d_str_mn = sdesc_sw128(warp_uniform(s_stream), C::kPanelBytes, 1024);
+      bool ok = mbar_wait_warp(res_full, 0, abort_flag);
       for (int j = 0; ok && j < n; ++j) {
         const int st = j % ST;
-        if (!mbar_wait(&full[st], (j / ST) & 1, abort_flag)) break;
+        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) break;
         tc_fence_after();
-        const uint32_t sa = s_stream + st * C::kStageBytes;
-        const uint32_t sb = sa + C::kBlockBytes;
-        ss_mma(tmem + 0, s_res_a, sa);      // S^T = K Q^T  |  S = Q K^T
-        ss_mma(tmem + 128, s_res_b, sb);    // dP^T = V dO^T |  dP = dO V^T
-        umma_commit(s_full);
-        if (!mbar_wait(p_full, j & 1, abort_flag)) break;
-        tc_fence_after();
-        if constexpr (kDKV) {
-          ts_mma(tmem + 256, tmem + 0, sb, j > 0);         // dV += P^T dO
-          ts_mma(tmem + 256 + D, tmem + 128, sa, j > 0);   // dK += dS^T Q
-        } else {
-          ts_mma(tmem + 256, tmem + 0, sa, j > 0);         // dQ += dS K
+        const uint32_t sa = (static_cast<uint32_t>(st) * C::kStageBytes) >> 4;
+        const uint32_t sb = sa + (C::kBlockBytes >> 4);
+        if (elect_one()) {
+          bwd_issue_ss<D>(tm + 0, d_res_a, d_str_k + sa);     // S^T = K Q^T  |  S = Q K^T
+          bwd_issue_ss<D>(tm + 128, d_res_b, d_str_k + sb);   // dP^T = V dO^T |  dP = dO V^T
+          umma_commit(s_full);
         }
-        umma_commit(&empty[st]);
-        if (j == n - 1) umma_commit(acc_full);
+        __syncwarp();
+        if (!mbar_wait_warp(p_full, j & 1, abort_flag)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          if (j > 0) {
+            if constexpr (kDKV) {
+              bwd_issue_ts<D, true>(tm + 256, tm + 0, d_str_mn + sb);       // dV += P^T dO
+              bwd_issue_ts<D, true>(tm + 256 + D, tm + 128, d_str_mn + sa); // dK += dS^T Q
+            } else {
+              bwd_issue_ts<D, true>(tm + 256, tm + 0, d_str_mn + sa);       // dQ += dS K
+            }
+          } else {
+            if constexpr (kDKV) {
+              bwd_issue_ts<D, false>(tm + 256, tm + 0, d_str_mn + sb);
+              bwd_issue_ts<D, false>(tm + 256 + D, tm + 128, d_str_mn + sa);
+            } else {
+              bwd_issue_ts<D, false>(tm + 256, tm + 0, d_str_mn + sa);
+            }
+          }
+          umma_commit(&empty[st]);
+          if (j == n - 1) umma_commit(acc_full);
+        }
+        __syncwarp();
       }
-      umma_commit(mma_done);
+      if (elect_one()) umma_commit(mma_done);
+      __syncwarp();
       mbar_wait_drain(mma_done, 0);
     }
   } else {

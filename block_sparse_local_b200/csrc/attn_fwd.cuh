@@ -264,6 +264,34 @@ __device__ __forceinline__ int raster_row(const FwdParams& p, int row) {
   return slice * g.S + ((tt * g.ct + it) * g.H + th * g.ch + ih) * g.W + tw * g.cw + iw;
 }
 
+// S_slot = Q_slot K^T over d (SS; K block in stage ks).  TMEM: S0 at column
+// 0, S1 at 128.  All operands warp-uniform, accumulate flags constant.
+template <int D, int SLOT>
+__device__ __forceinline__ void fwd_issue_s(uint32_t tm, uint64_t dq, uint64_t dk, int ks) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false);
+  const uint64_t qa = dq + ((SLOT * C::kBlockBytes) >> 4);
+  const uint64_t ka = dk + ((static_cast<uint32_t>(ks) * C::kBlockBytes) >> 4);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
+    umma_ss(tm + SLOT * 128u, qa + off, ka + off, kIdesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// O_slot (+)= P_slot V (TS: P from the first 64 columns of S_slot in TMEM,
+// V block in stage vs as an MN-major operand, N = d).
+template <int D, int SLOT, bool ACC>
+__device__ __forceinline__ void fwd_issue_pv(uint32_t tm, uint64_t dv, int vs) {
+  using C = FwdCfg<D>;
+  constexpr uint32_t kIdesc = idesc_bf16(kBM, D, true);
+  const uint64_t va = dv + ((static_cast<uint32_t>(vs) * C::kBlockBytes) >> 4);
+#pragma unroll
+  for (int kk = 0; kk < kBN / 16; ++kk)
+    umma_ts(tm + C::kOCol + SLOT * D, tm + SLOT * 128u + kk * 8, va + ((kk * 16 * 128) >> 4),
+            kIdesc, (ACC || kk > 0) ? 1u : 0u);
+}
+
 template <int D, Mode M, bool R>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
@@ -381,73 +409,75 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && !skip) {
-      constexpr uint32_t kIdescQK = idesc_bf16(kBM, kBN, false);
-      constexpr uint32_t kIdescPV = idesc_bf16(kBM, D, true);
-      auto t_s = [&](int slot) { return tmem + (slot ? 128u : 0u); };
-      auto t_o = [&](int slot) { return tmem + C::kOCol + (slot ? uint32_t(D) : 0u); };
-      auto issue_s = [&](int slot, int ks) {
-        const uint32_t qa = smem_q + slot * C::kBlockBytes;
-        const uint32_t ka = smem_k + ks * C::kBlockBytes;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kPanelBytes + (kk & 3) * 32;
-          umma_ss(t_s(slot), sdesc_sw128(qa + off, 16, 1024),
-                  sdesc_sw128(ka + off, 16, 1024), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int slot, int vs, bool acc) {
-        const uint32_t va = smem_v + vs * C::kBlockBytes;
-#pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_ts(t_o(slot), t_s(slot) + kk * 8,
-                  sdesc_sw128(va + kk * 16 * 128, C::kPanelBytes, 1024), kIdescPV,
-                  (acc || kk > 0) ? 1u : 0u);
-        }
-      };
-      bool ok = mbar_wait(q_full, 0, abort_flag) && mbar_wait(&k_full[0], 0, abort_flag);
+    // The whole warp runs the loop and waits; one elected lane issues (the
+    // same lane every time, so the MMAs and commits keep their issue order).
+    if (!skip) {
+      const uint32_t tm = warp_uniform(tmem);
+      // descriptor bases; per-MMA offsets go into the address field (bytes >> 4)
+      const uint64_t dq = sdesc_sw128(warp_uniform(smem_q), 16, 1024);
+      const uint64_t dk = sdesc_sw128(warp_uniform(smem_k), 16, 1024);
+      const uint64_t dv = sdesc_sw128(warp_uniform(smem_v), C::kPanelBytes, 1024);
+      bool ok = mbar_wait_warp(q_full, 0, abort_flag) && mbar_wait_warp(&k_full[0], 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_s(0, 0);
-        umma_commit(&s_full[0]);
-        if (two) {
-          issue_s(1, 0);
-          umma_commit(&s_full[1]);
+        if (elect_one()) {
+          fwd_issue_s<D, 0>(tm, dq, dk, 0);
+          umma_commit(&s_full[0]);
+          if (two) {
+            fwd_issue_s<D, 1>(tm, dq, dk, 0);
+            umma_commit(&s_full[1]);
+          }
+          umma_commit(&k_empty[0]);
         }
-        umma_commit(&k_empty[0]);
+        __syncwarp();
         for (int j = 0; j < n; ++j) {
           const int vs = j % VST;
           const int jn = j + 1;
           const int ksn = jn % KST;
-          if (!mbar_wait(&p_full[0], j & 1, abort_flag)) break;
-          if (!mbar_wait(&v_full[vs], (j / VST) & 1, abort_flag)) break;
+          if (!mbar_wait_warp(&p_full[0], j & 1, abort_flag)) break;
+          if (!mbar_wait_warp(&v_full[vs], (j / VST) & 1, abort_flag)) break;
           tc_fence_after();
-          issue_pv(0, vs, j > 0);
+          if (elect_one()) {
+            if (j > 0) fwd_issue_pv<D, 0, true>(tm, dv, vs);
+            else fwd_issue_pv<D, 0, false>(tm, dv, vs);
+          }
+          __syncwarp();
           if (jn < n) {
-            if (!mbar_wait(&k_full[ksn], (jn / KST) & 1, abort_flag)) break;
+            if (!mbar_wait_warp(&k_full[ksn], (jn / KST) & 1, abort_flag)) break;
             tc_fence_after();
-            issue_s(0, ksn);
-            umma_commit(&s_full[0]);
-          } else {
+            if (elect_one()) {
+              fwd_issue_s<D, 0>(tm, dq, dk, ksn);
+              umma_commit(&s_full[0]);
+            }
+          } else if (elect_one()) {
             umma_commit(&o_full[0]);
           }
+          __syncwarp();
           if (two) {
-            if (!mbar_wait(&p_full[1], j & 1, abort_flag)) break;
+            if (!mbar_wait_warp(&p_full[1], j & 1, abort_flag)) break;
             tc_fence_after();
-            issue_pv(1, vs, j > 0);
-            if (jn < n) {
-              issue_s(1, ksn);
-              umma_commit(&s_full[1]);
-            } else {
-              umma_commit(&o_full[1]);
+            if (elect_one()) {
+              if (j > 0) fwd_issue_pv<D, 1, true>(tm, dv, vs);
+              else fwd_issue_pv<D, 1, false>(tm, dv, vs);
+              if (jn < n) {
+                fwd_issue_s<D, 1>(tm, dq, dk, ksn);
+                umma_commit(&s_full[1]);
+              } else {
+                umma_commit(&o_full[1]);
+              }
             }
+            __syncwarp();
           }
-          umma_commit(&v_empty[vs]);
-          if (jn < n) umma_commit(&k_empty[ksn]);
+          if (elect_one()) {
+            umma_commit(&v_empty[vs]);
+            if (jn < n) umma_commit(&k_empty[ksn]);
+          }
+          __syncwarp();
         }
       }
       // No MMA may still run when TMEM is released.
-      umma_commit(mma_done);
+      if (elect_one()) umma_commit(mma_done);
+      __syncwarp();
       mbar_wait_drain(mma_done, 0);
     }
   } else {

@@ -167,6 +167,28 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return p;
 }
 
+// ---------------------------------------------------------------- issue helpers
+// tcgen05.mma issues at the tensor pipe's full rate only when its operands
+// (addresses, descriptors, the accumulate flag) are warp-uniform values the
+// compiler can see as such; an operand that changes every iteration in a
+// per-thread register roughly halves the issue rate of a 128x128x16 MMA.  So
+// MMA roles run as whole warps: bases are broadcast with warp_uniform(), loop
+// counters are warp-uniform, accumulate flags are compile-time constants, and
+// one lane chosen by elect_one() issues.
+__device__ __forceinline__ uint32_t warp_uniform(uint32_t x) {
+  return __shfl_sync(0xffffffffu, x, 0);
+}
+
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile(
