@@ -23,7 +23,7 @@ __all__ = [
     "retained_pairs", "STATUS", "forward_noalloc", "forward_raster", "swa3d_forward",
     "hilbert_reorder", "build_slide_block_lists", "slide2d_forward", "slide_attention_2d",
     "backward", "SlidingTileAttentionFunction", "TileReorderFunction",
-    "sliding_tile_attention_host",
+    "sliding_tile_attention_host", "use_pair_kernel",
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
@@ -35,7 +35,7 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
             "sta_swa3d_forward", "sta_debug_inject", "sta_hilbert_reorder",
             "sta_build_slide_block_lists", "sta_slide2d_forward", "sta_backward",
-            "sta_forward_raster_host")
+            "sta_forward_raster_host", "sta_debug_pair_kernel")
 
 
 class StaError(RuntimeError):
@@ -77,6 +77,7 @@ def lib():
     L.sta_swa_forward.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P]
     L.sta_device_status.argtypes = [_P]
     L.sta_debug_inject.argtypes = [_I, _I]
+    L.sta_debug_pair_kernel.argtypes = [_I]
     L.sta_backward.argtypes = [_P] * 9 + fwd
     L.sta_hilbert_reorder.argtypes = [_P, _P, _I, _I, _I, _I, _I, _P]
     L.sta_build_slide_block_lists.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P]
@@ -410,6 +411,12 @@ def swa_forward(q, k, v, window, causal=True, out=None):
                                  int(window), int(bool(causal)), _stream(q)),
            "sta_swa_forward")
     return out
+
+
+def use_pair_kernel(pair=True):
+    """Kernel selection hook for the d = 128 STA forward: CTA pairs
+    (pair=True) or the one-SM kernel (pair=False, the library default)."""
+    _check(lib().sta_debug_pair_kernel(int(bool(pair))), "sta_debug_pair_kernel")
 
 
 def device_status(device=None):

@@ -14,24 +14,25 @@
 //    positions as on the sliding-window search-result page).  Blocks cut by
 //    the band edges are masked per element.
 //
-// CTA = 10 warps, one work item = up to two 128-row query blocks that read
-// the same key blocks:
+// CTA = 2 + 8 * kSplit warps (18 with kSplit = 2), one work item = up to
+// two 128-row query blocks ("slots") that read the same key blocks:
 //   warp 0      TMA producer (one thread): Q once, then K and V blocks into
 //               K / V rings of shared-memory stages (128-byte swizzle).
-//   warp 1      MMA issuer (one thread) and TMEM owner:
-//               S_i = Q_i K^T (SS, M=128 N=128 K=d), O_i += P_i V (TS: P
-//               from TMEM, V from shared memory, N=d), ping-ponging the two
-//               slots so the tensor pipe works on one slot while the other
-//               slot's softmax runs.
-//   warps 2-5   softmax of slot 0, warps 6-9 softmax of slot 1: one thread
-//               per query row (TMEM lane), reads its 128 scores, updates the
-//               running max / sum, writes bf16 P over the first 64 columns
-//               of S, rescales its O row when the max grew by more than
-//               2^8, and finally normalises O and stores it.
+//   warp 1      MMA issuer (the whole warp waits, one elected lane issues)
+//               and TMEM owner: S_i = Q_i K^T (SS, M=128 N=128 K=d),
+//               O_i += P_i V (TS: P from TMEM, V from shared memory, N=d),
+//               ping-ponging the two slots so the tensor pipe works on one
+//               slot while the other slot's softmax runs.
+//   warps 2..   softmax, 4 * kSplit warps per slot: kSplit warps share each
+//               query row (TMEM lane), each with 128 / kSplit of its scores;
+//               they update the running max / sum, write bf16 P over the
+//               first half of their own score columns, rescale their O
+//               columns when the max grew by more than 2^8, and finally
+//               normalise O and store it.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
-// O1 [256+d, 256+2d); P_i aliases the first 64 columns of S_i.  The MMA that
-// overwrites S_i with the next scores is issued after the P_i.V MMA that
-// reads P_i; tcgen05 MMAs of one thread execute in issue order.
+// O1 [256+d, 256+2d); P_i aliases half of S_i.  The MMA that overwrites S_i
+// with the next scores is issued after the P_i.V MMA that reads P_i;
+// tcgen05 MMAs of one thread execute in issue order.
 #pragma once
 
 #include "device_ptx.cuh"
@@ -46,6 +47,7 @@ constexpr int kBN = 128;        // keys per block
 #define STA_SOFTMAX_SPLIT 2
 #endif
 constexpr int kSplit = STA_SOFTMAX_SPLIT;
+
 constexpr int kFwdThreads = 64 + 256 * kSplit;
 constexpr int kWarpTma = 0;
 constexpr int kWarpMma = 1;
@@ -74,6 +76,7 @@ struct RasterGeom {
 
 struct FwdParams {
   const WorkItem* items;
+  const int* item_off;  // CTA pairs: items of cluster c are [item_off[c], item_off[c + 1])
   const int* counts;
   const int* ids;
   int max_k;
@@ -88,6 +91,8 @@ struct FwdParams {
   const uint32_t* coords;  // kSlide2d: x | y << 16 of every position of the order
   int grid_n;         // kSlide2d: n of the n x n grid
   int win2;           // kSlide2d: w of the w x w window
+  int khalf_t;        // CTA pairs, raster order: key halves split along t (1) or h (0)
+  int kbox_t, kbox_h; // CTA pairs, raster order: the 128-row block's box along t, h
   float scale_log2;   // log2(e) / sqrt(d)
   __nv_bfloat16* out;
   float* lse;
@@ -279,17 +284,23 @@ __device__ __forceinline__ void fwd_issue_s(uint32_t tm, uint64_t dq, uint64_t d
   }
 }
 
-// O_slot (+)= P_slot V (TS: P from the first 64 columns of S_slot in TMEM,
-// V block in stage vs as an MN-major operand, N = d).
+// O_slot (+)= P_slot V (TS: P from TMEM, V block in stage vs as an MN-major
+// operand, N = d).  P of the keys served by softmax column group g (128 /
+// kSplit keys each) sits in the first half of that group's own score
+// columns: keys 16 kk .. 16 kk + 15 at column (kk / G) * 128 / kSplit +
+// (kk % G) * 8 of S_slot, G = 8 / kSplit k-steps per group.
 template <int D, int SLOT, bool ACC>
 __device__ __forceinline__ void fwd_issue_pv(uint32_t tm, uint64_t dv, int vs) {
   using C = FwdCfg<D>;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, D, true);
+  constexpr int G = (kBN / 16) / kSplit;
   const uint64_t va = dv + ((static_cast<uint32_t>(vs) * C::kBlockBytes) >> 4);
 #pragma unroll
-  for (int kk = 0; kk < kBN / 16; ++kk)
-    umma_ts(tm + C::kOCol + SLOT * D, tm + SLOT * 128u + kk * 8, va + ((kk * 16 * 128) >> 4),
+  for (int kk = 0; kk < kBN / 16; ++kk) {
+    const uint32_t acol = (kk / G) * (kBN / kSplit) + (kk % G) * 8;
+    umma_ts(tm + C::kOCol + SLOT * D, tm + SLOT * 128u + acol, va + ((kk * 16 * 128) >> 4),
             kIdesc, (ACC || kk > 0) ? 1u : 0u);
+  }
 }
 
 template <int D, Mode M, bool R>
@@ -338,7 +349,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&o_full[i], 1);
     }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], 32 * kSplit);
+    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], kSplit);   // one arrival per warp
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
     fence_mbar_init();
   }
@@ -434,8 +445,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const int vs = j % VST;
           const int jn = j + 1;
           const int ksn = jn % KST;
-          if (!mbar_wait_warp(&p_full[0], j & 1, abort_flag)) break;
+          // V arrives long before P: wait for it first, so the wait for P
+          // is the last thing between the softmax and the P.V MMA
           if (!mbar_wait_warp(&v_full[vs], (j / VST) & 1, abort_flag)) break;
+          if (!mbar_wait_warp(&p_full[0], j & 1, abort_flag)) break;
           tc_fence_after();
           if (elect_one()) {
             if (j > 0) fwd_issue_pv<D, 0, true>(tm, dv, vs);
@@ -501,7 +514,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (!skip && (slot == 0 || two)) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
       const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u) + half * kCols;
-      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u) + half * (kCols / 2);
+      // P over the first half of this thread's own score columns, so no
+      // warp overwrites scores that another warp has still to read
+      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u) + half * kCols;
       const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0) + half * kOCols;
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY;   // running max, log2 units of the scaled scores
@@ -592,19 +607,44 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
               if (!((km >> c) & 1ull)) s[c] = -INFINITY;
           }
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max: four independent chains of three-input max
+        constexpr int kQ = kCols / 4;
+        float mq[4];
 #pragma unroll
-        for (int c = 4; c < kCols; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int k4 = 0; k4 < 4; ++k4) {
+          float m = s[k4 * kQ];
+#pragma unroll
+          for (int i = 1; i + 1 < kQ; i += 2) m = fmax3(m, s[k4 * kQ + i], s[k4 * kQ + i + 1]);
+          if constexpr (kQ % 2 == 0) m = fmaxf(m, s[k4 * kQ + kQ - 1]);
+          mq[k4] = m;
         }
-        float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        // The two halves of a row must agree on the reference of the
+        // exponent.  Each half posts its max and goes on with a provisional
+        // reference (the running max, or its own max when that escalates past
+        // the running max by more than 2^8); the partner's max is read only
+        // after the exponentials, and the rare half whose reference was too
+        // low rescales its 64 values.  The exchange latency thus overlaps the
+        // exp2 work instead of sitting in front of it.
+        float* rb = red + ((j & 1) * 2 + slot) * 2 * kBM;
         if constexpr (kSplit == 2) {
-          float* rb = red + ((j & 1) * 2 + slot) * 2 * kBM;
           rb[half * kBM + r] = mx;
-          mbar_arrive(xb);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xb);
+        }
+        const float m_loc = mx * sl2;
+        const float m_prov = m_loc > m_run + 8.0f ? m_loc : m_run;
+        const float neg_p = (m_prov == -INFINITY) ? 0.f : -m_prov;
+        // exp2 of the scaled, shifted scores, in place
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 2) {
+          s[c] = fast_exp2(fmaf(s[c], sl2, neg_p));
+          s[c + 1] = fast_exp2(fmaf(s[c + 1], sl2, neg_p));
+          ls0 += s[c];
+          ls1 += s[c + 1];
+        }
+        if constexpr (kSplit == 2) {
           if (!mbar_wait_warp(xb, j & 1, abort_flag)) { done = false; break; }
           mx = fmaxf(mx, rb[(half ^ 1) * kBM + r]);
         }
@@ -616,20 +656,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           m_run = m_cand;
           l_run *= alpha;
         }
-        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-        // exp2 of the scaled, shifted scores -> bf16 P in TMEM
-        float ls0 = 0.f, ls1 = 0.f;
+        if (m_run > m_prov) {
+          const float corr = fast_exp2(m_prov - m_run);
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) s[c] *= corr;
+          ls0 *= corr;
+          ls1 *= corr;
+        }
+        // bf16 P over the first half of this thread's own score columns
 #pragma unroll
         for (int cc = 0; cc < kCols / 32; ++cc) {
           uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(s[cc * 32 + 2 * e], sl2, neg_m));
-            const float p1 = fast_exp2(fmaf(s[cc * 32 + 2 * e + 1], sl2, neg_m));
-            ls0 += p0;
-            ls1 += p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(s[cc * 32 + 2 * e], s[cc * 32 + 2 * e + 1]);
           STA_TMEM_ST16(t_p + cc * 16, pk);
         }
         l_run += ls0 + ls1;
@@ -655,7 +694,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if constexpr (kSplit == 2) {
           float* rb = red + ((n & 1) * 2 + slot) * 2 * kBM;
           rb[half * kBM + r] = l_run;
-          mbar_arrive(xb);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(xb);
           ok = mbar_wait_warp(xb, n & 1, abort_flag);
           if (ok) l_run += rb[(half ^ 1) * kBM + r];
         }

@@ -12,6 +12,7 @@
 #include <cstring>
 #include <map>
 #include <mutex>
+#include <queue>
 #include <string>
 #include <vector>
 
@@ -20,6 +21,7 @@
 #include "reorder.cuh"
 #include "tile_lists.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_pair.cuh"
 #include "hilbert.cuh"
 #include "attn_bwd.cuh"
 
@@ -84,13 +86,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [rows, d] bf16 row-major, box of 128 rows x 64 columns, 128-byte swizzle.
-sta_status make_row_map(CUtensorMap* map, const void* base, int64_t rows, int d) {
+// [rows, d] bf16 row-major, box of box_rows rows x 64 columns, 128-byte swizzle.
+sta_status make_row_map(CUtensorMap* map, const void* base, int64_t rows, int d,
+                        int box_rows = 128) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return STA_ERR_CUDA;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
-  cuuint32_t box[2] = {64, 128};
+  cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -252,6 +255,7 @@ struct Workspace {
   size_t cap = 0;
   std::string plan_key;     // key of the plan currently resident in `buf`
   std::vector<WorkItem> items;
+  std::vector<int> item_off;  // CTA-pair plans: first item of each cluster, + end
 };
 Workspace g_ws[64];
 
@@ -349,6 +353,36 @@ std::vector<WorkItem> plan_sta(const Geom& g, const Classes& cls, int B, int hea
   return items;
 }
 
+// Persistent CTA-pair kernel: items (sorted longest first) go, one at a time,
+// to the cluster with the least work so far (longest-processing-time-first);
+// equal lengths thus go round robin, so clusters running at the same time
+// work on neighbouring items.  Returns the items cluster by cluster and, in
+// *off, the first item of each cluster followed by the total.
+std::vector<WorkItem> assign_to_clusters(const std::vector<WorkItem>& items,
+                                         const std::vector<int>& lengths, int nclusters,
+                                         std::vector<int>* off) {
+  const int nc = std::max(1, std::min(nclusters, static_cast<int>(items.size())));
+  std::vector<std::vector<int>> per(nc);
+  using Load = std::pair<int64_t, int>;
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> heap;
+  for (int c = 0; c < nc; ++c) heap.push({0, c});
+  for (size_t i = 0; i < items.size(); ++i) {
+    Load l = heap.top();
+    heap.pop();
+    per[l.second].push_back(static_cast<int>(i));
+    l.first += lengths[i];
+    heap.push(l);
+  }
+  std::vector<WorkItem> out;
+  out.reserve(items.size());
+  off->assign(1, 0);
+  for (int c = 0; c < nc; ++c) {
+    for (int i : per[c]) out.push_back(items[i]);
+    off->push_back(static_cast<int>(out.size()));
+  }
+  return out;
+}
+
 std::string sta_key(int dev, int B, int heads, int d, const Geom& g, const int* window) {
   std::string k = "sta:" + std::to_string(dev) + ":" + std::to_string(B) + ":" +
                   std::to_string(heads) + ":" + std::to_string(d) + ":" + std::to_string(g.T) +
@@ -380,6 +414,46 @@ sta_status launch_attn(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
+
+// The d = 128 STA kernel on CTA pairs (attn_fwd_pair.cuh): one cluster of two
+// CTAs per work item.
+template <bool R>
+sta_status launch_attn_pair(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                            const FwdParams& prm, int num_items, cudaStream_t st,
+                            const CUtensorMap* mq5, const CUtensorMap* mk5,
+                            const CUtensorMap* mv5) {
+  constexpr int smem = sta::PairCfg::kSmemBytes;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  STA_CUDA_TRY(cudaGetDevice(&dev));
+  if (!attr_set[dev]) {
+    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_fwd_pair_kernel<R>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * static_cast<unsigned>(num_items), 1, 1);
+  cfg.blockDim = dim3(sta::kPairThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  STA_CUDA_TRY(cudaLaunchKernelEx(&cfg, sta::attn_fwd_pair_kernel<R>, mq, mk, mv,
+                                  mq5 ? *mq5 : mq, mk5 ? *mk5 : mk, mv5 ? *mv5 : mv, prm));
+  return STA_OK;
+}
+
+// Kernel choice for d = 128 STA: 0 = the one-SM kernel (the default; also
+// the kernel of d = 64 and of the masked modes), 1 = the CTA-pair kernel
+// when the geometry allows (opt-in: on the video+text workload it is as fast
+// on tile-ordered inputs and slower on raster-ordered ones, its K / V loads
+// taking longer to land than its three score buffers cover).
+int g_pair_mode = 0;
 
 sta_status forward_impl(const void* q, const void* k, const void* v, void* out, float* lse,
                         int B, int heads, int d, int T, int H, int W, const int tile[3],
@@ -448,26 +522,49 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   const size_t counts_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
   const size_t ids_bytes = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
 
-  const std::string key = (token_mode ? "tok:" : "") + sta_key(dev, B, heads, d, g, window);
+  // CTA pairs (attn_fwd_pair.cuh) for d = 128 STA; in raster order each CTA
+  // loads 64-row halves of the key blocks, so a block's box must split into
+  // two boxes (along t, else along h).
+  const bool khalf_t = box_t >= 2;
+  const bool pair = g_pair_mode == 1 && d == 128 && !token_mode &&
+                    (!raster || khalf_t || box_h % 2 == 0);
+  const int nclusters_max = std::max(1, g_dev[dev].num_sms / 2);
+
+  const std::string key = std::string(token_mode ? "tok:" : "") + (pair ? "pair:" : "") +
+                          sta_key(dev, B, heads, d, g, window);
   Workspace& ws = g_ws[dev];
   std::vector<WorkItem> fresh;
+  std::vector<int> fresh_off;
   const bool cached = (ws.plan_key == key && ws.buf != nullptr);
-  if (!cached) fresh = plan_sta(g, cls, B, heads, max_k, nullptr, token_mode);
+  if (!cached) {
+    std::vector<int> lengths;
+    fresh = plan_sta(g, cls, B, heads, max_k, &lengths, token_mode);
+    if (pair) fresh = assign_to_clusters(fresh, lengths, nclusters_max, &fresh_off);
+  }
   const std::vector<WorkItem>& items = cached ? ws.items : fresh;
-  const size_t items_bytes = sizeof(WorkItem) * items.size();
-  s = ensure_workspace(dev, counts_bytes + ids_bytes + items_bytes);
+  const std::vector<int>& offs = cached ? ws.item_off : fresh_off;
+  const size_t items_bytes = align_up(sizeof(WorkItem) * items.size(), 256);
+  const size_t off_bytes = sizeof(int) * offs.size();
+  s = ensure_workspace(dev, counts_bytes + ids_bytes + items_bytes + off_bytes);
   if (s != STA_OK) return s;
   uint8_t* wbuf = static_cast<uint8_t*>(ws.buf);
   int* d_counts = reinterpret_cast<int*>(wbuf);
   int* d_ids = reinterpret_cast<int*>(wbuf + counts_bytes);
   WorkItem* d_items = reinterpret_cast<WorkItem*>(wbuf + counts_bytes + ids_bytes);
+  int* d_off = reinterpret_cast<int*>(wbuf + counts_bytes + ids_bytes + items_bytes);
   if (ws.plan_key != key) {
     ws.items = std::move(fresh);
+    ws.item_off = std::move(fresh_off);
     STA_CUDA_TRY(cudaMemcpyAsync(d_items, ws.items.data(), sizeof(WorkItem) * ws.items.size(),
                                  cudaMemcpyHostToDevice, st));
+    if (!ws.item_off.empty())
+      STA_CUDA_TRY(cudaMemcpyAsync(d_off, ws.item_off.data(), sizeof(int) * ws.item_off.size(),
+                                   cudaMemcpyHostToDevice, st));
     ws.plan_key = key;
   }
-  const int num_items = static_cast<int>(ws.items.size());
+  // one CTA per item, or (pairs) one persistent cluster per item list
+  const int num_items = pair ? static_cast<int>(ws.item_off.size()) - 1
+                             : static_cast<int>(ws.items.size());
 
   CUtensorMap mq, mk, mv;
   s = make_row_map(&mq, q, total_rows, d);
@@ -479,8 +576,9 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   launch_lists(d_counts, d_ids, cls, g, max_k, st, token_mode);
   STA_CUDA_TRY(cudaGetLastError());
 
-  FwdParams prm;
+  FwdParams prm{};
   prm.items = d_items;
+  prm.item_off = pair ? d_off : nullptr;
   prm.counts = d_counts;
   prm.ids = d_ids;
   prm.max_k = max_k;
@@ -501,13 +599,26 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   prm.rg.T = g.T;
   if (token_mode)
     for (int a = 0; a < 3; ++a) prm.win3[a] = token_window[a];
+  prm.khalf_t = khalf_t ? 1 : 0;
+  prm.kbox_t = box_t;
+  prm.kbox_h = box_h;
+  CUtensorMap mk_half;
+  if (pair) {
+    s = make_row_map(&mk_half, k, total_rows, d, 64);
+    if (s != STA_OK) return s;
+  }
   if (raster) {
     CUtensorMap q5, k5, v5;
     const int slices = B * heads;
     s = make_raster_map(&q5, q, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
-    if (s == STA_OK) s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+    if (s == STA_OK && pair)
+      s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw,
+                          khalf_t ? box_h : box_h / 2, khalf_t ? box_t / 2 : box_t);
+    else if (s == STA_OK)
+      s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
     if (s == STA_OK) s = make_raster_map(&v5, v, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
     if (s != STA_OK) return s;
+    if (pair) return launch_attn_pair<true>(mq, mk_half, mv, prm, num_items, st, &q5, &k5, &v5);
     if (token_mode) {
       if (d == 128)
         return launch_attn<128, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5,
@@ -519,6 +630,8 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
     return launch_attn<64, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
   }
   if (token_mode) return STA_ERR_UNSUPPORTED;
+  if (pair) return launch_attn_pair<false>(mq, mk_half, mv, prm, num_items, st, nullptr, nullptr,
+                                           nullptr);
   if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
   return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
 }
@@ -804,8 +917,9 @@ sta_status forward_noalloc_impl(const void* q, const void* k, const void* v, voi
   launch_lists(d_counts, d_ids, cls, g, max_k, st);
   STA_CUDA_TRY(cudaGetLastError());
 
-  FwdParams prm;
+  FwdParams prm{};
   prm.items = d_items;
+  prm.item_off = nullptr;
   prm.counts = d_counts;
   prm.ids = d_ids;
   prm.max_k = max_k;
@@ -1206,7 +1320,7 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   if (s == STA_OK) s = make_row_map(&mk, k, int64_t(B) * hkv * S, d);
   if (s == STA_OK) s = make_row_map(&mv, v, int64_t(B) * hkv * S, d);
   if (s != STA_OK) return s;
-  FwdParams prm;
+  FwdParams prm{};
   std::memset(&prm, 0, sizeof(prm));
   prm.items = d_items;
   prm.window = window;
@@ -1216,6 +1330,13 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   const int num_items = static_cast<int>(ws.items.size());
   if (d == 128) return launch_attn<128, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
   return launch_attn<64, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
+}
+
+sta_status sta_debug_pair_kernel(int pair) {
+  if (pair != 0 && pair != 1) return STA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_mu);
+  g_pair_mode = pair;
+  return STA_OK;
 }
 
 sta_status sta_debug_inject(int mode, int wait_limit_ms) {
@@ -1336,7 +1457,7 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void
   if (s == STA_OK) s = make_row_map(&mk, k, rows, d);
   if (s == STA_OK) s = make_row_map(&mv, v, rows, d);
   if (s != STA_OK) return s;
-  FwdParams prm;
+  FwdParams prm{};
   std::memset(&prm, 0, sizeof(prm));
   prm.items = items;
   prm.counts = counts;

@@ -269,6 +269,19 @@ sta_status sta_device_status(void* stream);
  */
 sta_status sta_debug_inject(int mode, int wait_limit_ms);
 
+/*
+ * sta_debug_pair_kernel - kernel selection hook with no counterpart on the
+ * pages, for the d = 128 STA forward (sta_forward, sta_forward_lse,
+ * sta_forward_raster and the host-buffer form).  pair = 0 (the default): the
+ * one-SM kernel that d = 64 and the other modes use; pair = 1: a persistent
+ * cluster of two CTAs per pair of SMs, tcgen05 MMAs issued for both SMs at
+ * once (M = 256), each SM loading half of every key / value block, three
+ * score buffers in tensor memory.  Both compute the same function; the tests
+ * run both.  Host-side setting for the calling process; STA_ERR_INVALID_ARG
+ * for other values.
+ */
+sta_status sta_debug_pair_kernel(int pair);
+
 /* Static, never NULL. */
 const char* sta_status_string(sta_status s);
 
