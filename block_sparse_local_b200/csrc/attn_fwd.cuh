@@ -197,16 +197,16 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-// Loads one 128-row block whose first row in the tile-ordered view is `row`
-// (kPanels loads of 128 rows x 128 bytes).  Tile-ordered tensors and the text
-// block: rows of the 2-D [B*heads*S, d] view.  Video blocks of raster-ordered
-// tensors (R): the block is a box of its tile in the (d, W, H, T, slice) view;
-// the box lands in shared memory in the tile's own (t, h, w) order.
+// Loads one 64-column panel (128 rows x 128 bytes, 128-byte swizzle) of the
+// 128-row block whose first row in the tile-ordered view is `row`.
+// Tile-ordered tensors and the text block: rows of the 2-D [B*heads*S, d]
+// view.  Video blocks of raster-ordered tensors (R): the block is a box of its
+// tile in the (d, W, H, T, slice) view, landing in shared memory in the
+// tile's own (t, h, w) order.
 template <int D, bool R>
-__device__ __forceinline__ void load_block(uint8_t* dst, const CUtensorMap* m2,
+__device__ __forceinline__ void load_panel(uint8_t* dst, const CUtensorMap* m2,
                                            const CUtensorMap* m5, uint64_t* bar, int row,
-                                           const FwdParams& p, uint64_t pol) {
-  constexpr int kPanels = D / 64;
+                                           const FwdParams& p, uint64_t pol, int pn) {
   if constexpr (R) {
     const RasterGeom& g = p.rg;
     const int slice = row / g.S;
@@ -219,16 +219,12 @@ __device__ __forceinline__ void load_block(uint8_t* dst, const CUtensorMap* m2,
       const int tw = tile % g.NW;
       const int th = (tile / g.NW) % g.NH;
       const int tt = tile / (g.NW * g.NH);
-#pragma unroll
-      for (int pn = 0; pn < kPanels; ++pn)
-        tma_load_5d(dst + pn * 128 * 128, m5, bar, pn * 64, tw * g.cw, th * g.ch + ih,
-                    tt * g.ct + it, slice, pol);
+      tma_load_5d(dst + pn * 128 * 128, m5, bar, pn * 64, tw * g.cw, th * g.ch + ih,
+                  tt * g.ct + it, slice, pol);
       return;
     }
   }
-#pragma unroll
-  for (int pn = 0; pn < kPanels; ++pn)
-    tma_load_2d_hint(dst + pn * 128 * 128, m2, bar, pn * 64, row, pol);
+  tma_load_2d_hint(dst + pn * 128 * 128, m2, bar, pn * 64, row, pol);
 }
 
 // kSwa3d, tiles with 8 x 8 tokens per t-slice: each 128-key block holds two
@@ -376,46 +372,47 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && !skip) {
+    // A thread's TMA loads complete one after another, so each operand panel
+    // has its own lane: lanes 0 .. kPanels-1 load the key panels, lanes
+    // kPanels .. 2 kPanels-1 the value panels (and the first ones the query
+    // blocks); the panel-0 lane of each operand posts the expected bytes.
+    constexpr int kPanels = C::kPanels;
+    if (lane < 2 * kPanels && !skip) {
+      const bool is_v = lane >= kPanels;
+      const int pn = lane % kPanels;
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
       const bool drop_q = *reinterpret_cast<volatile int*>(&g_inject) == 1;
       if (!drop_q) {
-        mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
-        for (int s = 0; s < (two ? 2 : 1); ++s) {
-          const int qrow = s ? item.q1 : item.q0;
-          load_block<D, R>(smem + C::kQOff + s * C::kBlockBytes, &tmap_q, &tmap_q5, q_full,
-                           qrow, p, pol_q);
-        }
+        if (lane == 0) mbar_arrive_expect_tx(q_full, (two ? 2 : 1) * C::kBlockBytes);
+        const int s = is_v ? 1 : 0;      // key lanes load slot 0, value lanes slot 1
+        if (s == 0 || two)
+          load_panel<D, R>(smem + C::kQOff + s * C::kBlockBytes, &tmap_q, &tmap_q5, q_full,
+                           s ? item.q1 : item.q0, p, pol_q, pn);
       }
-      int issued = 0;
+      uint64_t* full = is_v ? v_full : k_full;
+      uint64_t* empty = is_v ? v_empty : k_empty;
+      constexpr int NST = KST;           // key and value rings have the same depth
+      static_assert(KST == VST, "one ring depth for both operands");
+      const CUtensorMap* m2 = is_v ? &tmap_v : &tmap_k;
+      const CUtensorMap* m5 = is_v ? &tmap_v5 : &tmap_k5;
+      uint8_t* base = smem + (is_v ? C::kVOff : C::kKOff);
       for (int j = 0; j < n; ++j) {
-        const int ks = j % KST;
-        if (j >= KST && !mbar_wait(&k_empty[ks], ((j / KST) - 1) & 1, abort_flag)) break;
+        const int st = j % NST;
+        if (j >= NST && !mbar_wait(&empty[st], ((j / NST) - 1) & 1, abort_flag)) break;
         const int row = seq_row<M>(p, seq, j);
-        mbar_arrive_expect_tx(&k_full[ks], C::kBlockBytes);
-        load_block<D, R>(smem + C::kKOff + ks * C::kBlockBytes, &tmap_k, &tmap_k5, &k_full[ks],
-                         row, p, pol_kv);
-        const int vs = j % VST;
-        if (j >= VST && !mbar_wait(&v_empty[vs], ((j / VST) - 1) & 1, abort_flag)) {
-          issued = j * 2 + 1;
-          break;
-        }
-        mbar_arrive_expect_tx(&v_full[vs], C::kBlockBytes);
-        load_block<D, R>(smem + C::kVOff + vs * C::kBlockBytes, &tmap_v, &tmap_v5, &v_full[vs],
-                         row, p, pol_kv);
-        issued = j * 2 + 2;
+        if (pn == 0) mbar_arrive_expect_tx(&full[st], C::kBlockBytes);
+        load_panel<D, R>(base + st * C::kBlockBytes, m2, m5, &full[st], row, p, pol_kv, pn);
       }
+      __syncwarp((1u << (2 * kPanels)) - 1u);
       // Leave no copy in flight: wait for the last load of every stage.
-      if (!drop_q) mbar_wait_drain(q_full, 0);
-      const int nk = (issued + 1) / 2, nv = issued / 2;
-      for (int s = 0; s < KST && s < nk; ++s) {
-        const int last = s + ((nk - 1 - s) / KST) * KST;
-        mbar_wait_drain(&k_full[s], (last / KST) & 1);
-      }
-      for (int s = 0; s < VST && s < nv; ++s) {
-        const int last = s + ((nv - 1 - s) / VST) * VST;
-        mbar_wait_drain(&v_full[s], (last / VST) & 1);
+      if (lane == 0) {
+        if (!drop_q) mbar_wait_drain(q_full, 0);
+        for (int st = 0; st < NST && st < n; ++st) {
+          const int last = st + ((n - 1 - st) / NST) * NST;
+          mbar_wait_drain(&k_full[st], (last / NST) & 1);
+          mbar_wait_drain(&v_full[st], (last / NST) & 1);
+        }
       }
     }
   } else if (warp == kWarpMma) {

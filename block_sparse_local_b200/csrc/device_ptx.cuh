@@ -460,24 +460,4 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// 2^x on the FMA and integer pipes, to take part of the softmax's
-// exponentials off the MUFU pipe (which alone runs at 16 per cycle per SM,
-// as fast as the tensor cores consume scores at d = 128).  Split
-// x = i + f with i = round(x) (adding 1.5 * 2^23 rounds to an integer in the
-// low mantissa bits) and f in [-1/2, 1/2]; 2^f by a cubic with minimax
-// relative error (Remez exchange, coefficients from gen_exp2_poly.py,
-// max relative error 7.5e-5, below the bf16 rounding of P); 2^i by adding
-// i to the exponent field.  x is clamped at -126 (masked scores are -inf):
-// 2^f >= 0.707 has biased exponent >= 126, so the sum stays a non-negative
-// float (a tiny or subnormal value, far below anything the bf16 P keeps).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(__uint_as_float(0x3d61fbb0u), f, __uint_as_float(0x3e786f0du));
-  p = fmaf(p, f, __uint_as_float(0x3f31798du));
-  p = fmaf(p, f, __uint_as_float(0x3f7ffb49u));
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 }  // namespace sta

@@ -539,7 +539,24 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   if (!cached) {
     std::vector<int> lengths;
     fresh = plan_sta(g, cls, B, heads, max_k, &lengths, token_mode);
-    if (pair) fresh = assign_to_clusters(fresh, lengths, nclusters_max, &fresh_off);
+    if (pair) {
+      // slice-major (longest first within a slice), so that the clusters
+      // running at the same time read the keys / values of one or two heads
+      std::vector<int> idx(fresh.size());
+      for (size_t i = 0; i < idx.size(); ++i) idx[i] = static_cast<int>(i);
+      std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) {
+        const int sa = fresh[a].kv_base / g.S, sb = fresh[b].kv_base / g.S;
+        if (sa != sb) return sa < sb;
+        return lengths[a] > lengths[b];
+      });
+      std::vector<WorkItem> by_slice;
+      std::vector<int> len_by_slice;
+      for (int i : idx) {
+        by_slice.push_back(fresh[i]);
+        len_by_slice.push_back(lengths[i]);
+      }
+      fresh = assign_to_clusters(by_slice, len_by_slice, nclusters_max, &fresh_off);
+    }
   }
   const std::vector<WorkItem>& items = cached ? ws.items : fresh;
   const std::vector<int>& offs = cached ? ws.item_off : fresh_off;
