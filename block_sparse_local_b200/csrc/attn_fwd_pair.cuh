@@ -208,7 +208,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     mbar_init(o_free, 32);            // 16 softmax warps in each CTA
     mbar_init(mma_done, 1);
     for (int i = 0; i < 8; ++i) mbar_init(&xb[i], 2);   // one arrival per warp
-    for (int i = 0; i < 2; ++i) mbar_init(&ref_bar[i], 4);
+    // all 8 warps of the posting group: the half-0 warps after writing the
+    // value, the half-1 warps after reading the previous one, so the next
+    // writer of the slot cannot overtake a reader
+    for (int i = 0; i < 2; ++i) mbar_init(&ref_bar[i], 8);
     mbar_init(sum_bar, 16);
     *abort_flag = (error_raised() || it1 <= it0) ? 1 : 0;
     fence_mbar_init();
@@ -499,22 +502,24 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) mbar_arrive(xbg);
         if (!mbar_wait_warp(xbg, par, abort_flag)) { done = false; break; }
         mx = fmaxf(mx, rb[(half ^ 1) * 128 + r]);
-        // reference after the item's previous block (the other group's)
+        // reference after the item's previous block (the other group's).
+        // Every block but the cluster's first waits for the previous block's
+        // post, even the first block of an item, which does not use it: its
+        // own post reuses that slot and barrier, which the previous item's
+        // last block may still have to read.
         float m_prev = -INFINITY;
-        if (j > 0) {
+        if (g > 0) {
           if (!mbar_wait_warp(&ref_bar[(g - 1) & 1], ((g - 1) >> 1) & 1, abort_flag)) {
             done = false;
             break;
           }
-          m_prev = ref[((g - 1) & 1) * 128 + r];
+          if (j > 0) m_prev = ref[((g - 1) & 1) * 128 + r];
         }
         const float m_cand = mx * sl2;
         const float m_use = m_cand > m_prev + 8.0f ? m_cand : m_prev;
-        if (half == 0) {
-          ref[(g & 1) * 128 + r] = m_use;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ref_bar[g & 1]);
-        }
+        if (half == 0) ref[(g & 1) * 128 + r] = m_use;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ref_bar[g & 1]);
         if (m_g != m_use) {
           l_g = (m_g == -INFINITY) ? 0.f : l_g * fast_exp2(m_g - m_use);
           m_g = m_use;

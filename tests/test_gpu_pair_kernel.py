@@ -104,3 +104,21 @@ def test_pair_kernel_full_video_text_workload():
                                               rows=rows)
         err = np.abs(out[0, h].float().cpu().numpy()[rows] - want)
         assert err.max() <= MAX_ABS and err.mean() <= MEAN_ABS, (h, err.max(), err.mean())
+
+
+def test_pair_kernel_many_items_per_cluster():
+    # 2 x 8 slices of a 2 x 2 x 3 tile grid: ~300 work items, several per
+    # persistent cluster, so the pipeline runs across item boundaries
+    wins = [(1, 1, 1), (2, 2, 3), (1, 2, 2), (2, 1, 3)] * 2
+    w = workloads.small_sta_case(12, 16, 24, (6, 8, 8), wins, 77, True, d=128, B=2, seed=29)
+    shape = (w.T, w.H, w.W)
+    q, k, v = workloads.sta_inputs(w)
+    out = sta.forward_raster(q.cuda(), k.cuda(), v.cuda(), w.windows, w.text_len, w.has_text,
+                             shape, w.tile)
+    sta.device_status()
+    _compare(out.float().cpu().numpy(), _oracle(w, q, k, v))
+    sta.use_pair_kernel(False)
+    ref = sta.forward_raster(q.cuda(), k.cuda(), v.cuda(), w.windows, w.text_len, w.has_text,
+                             shape, w.tile)
+    sta.device_status()
+    assert (out.float() - ref.float()).abs().max().item() <= MAX_ABS
