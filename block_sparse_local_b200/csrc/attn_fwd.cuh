@@ -35,6 +35,8 @@
 // tcgen05 MMAs of one thread execute in issue order.
 #pragma once
 
+#include <type_traits>
+
 #include "device_ptx.cuh"
 
 namespace sta {
@@ -557,118 +559,157 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
-        uint32_t sr[kCols];
-#pragma unroll
-        for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_LD32(t_s + cc * 32, (sr + cc * 32));
-        tmem_wait_ld();
         float s[kCols];
+        // this thread's raw scores of block j, masked (called again by the
+        // rare recompute below: the scores stay in TMEM until P is stored)
+        auto load_scores = [&]() {
+          uint32_t sr[kCols];
 #pragma unroll
-        for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
-        int lo, hi;
-        if (seq_mask<M>(p, seq, j, r, lo, hi)) {
-          lo -= half * kCols;
-          hi -= half * kCols;
+          for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_LD32(t_s + cc * 32, (sr + cc * 32));
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < kCols; ++c)
-            if (c < lo || c >= hi) s[c] = -INFINITY;
-        }
-        if constexpr (M == Mode::kSlide2d) {
-          // per-element 2-D window test against the keys' grid coordinates
-          const uint4* kc = reinterpret_cast<const uint4*>(
-              p.coords + static_cast<size_t>(seq.ids[j]) * kBN + half * kCols);
-#pragma unroll
-          for (int c4 = 0; c4 < kCols / 4; ++c4) {
-            const uint4 v4 = __ldg(kc + c4);
-            const uint32_t cv[4] = {v4.x, v4.y, v4.z, v4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t dx = (cv[e] & 0xffffu) - static_cast<uint32_t>(sxlo);
-              const uint32_t dy = (cv[e] >> 16) - static_cast<uint32_t>(sylo);
-              if (dx >= static_cast<uint32_t>(swe) || dy >= static_cast<uint32_t>(swe))
-                s[c4 * 4 + e] = -INFINITY;
+          for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
+          int lo, hi;
+          if (seq_mask<M>(p, seq, j, r, lo, hi)) {
+            lo -= half * kCols;
+            hi -= half * kCols;
+  #pragma unroll
+            for (int c = 0; c < kCols; ++c)
+              if (c < lo || c >= hi) s[c] = -INFINITY;
+          }
+          if constexpr (M == Mode::kSlide2d) {
+            // per-element 2-D window test against the keys' grid coordinates
+            const uint4* kc = reinterpret_cast<const uint4*>(
+                p.coords + static_cast<size_t>(seq.ids[j]) * kBN + half * kCols);
+  #pragma unroll
+            for (int c4 = 0; c4 < kCols / 4; ++c4) {
+              const uint4 v4 = __ldg(kc + c4);
+              const uint32_t cv[4] = {v4.x, v4.y, v4.z, v4.w};
+  #pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const uint32_t dx = (cv[e] & 0xffffu) - static_cast<uint32_t>(sxlo);
+                const uint32_t dy = (cv[e] >> 16) - static_cast<uint32_t>(sylo);
+                if (dx >= static_cast<uint32_t>(swe) || dy >= static_cast<uint32_t>(swe))
+                  s[c4 * 4 + e] = -INFINITY;
+              }
             }
           }
-        }
-        if constexpr (M == Mode::kSwa3d) {
-          static_assert(kSplit == 2, "the 3-D window mask gives each half one t-slice");
-          if (tok_row && j < seq.nvid) {
-            const RasterGeom& g = p.rg;
-            const int kt = j / p.tile_blocks;
-            const int sb = j - kt * p.tile_blocks;
-            const int kid = seq.ids[kt];
-            const int ktw = kid % g.NW, kth = (kid / g.NW) % g.NH, ktt = kid / (g.NW * g.NH);
-            const uint64_t km = swa3d_half_mask(ktt * g.ct + sb * 2 + half, kth * g.ch,
-                                                ktw * g.cw, tws, twe);
-#pragma unroll
-            for (int c = 0; c < kCols; ++c)
-              if (!((km >> c) & 1ull)) s[c] = -INFINITY;
+          if constexpr (M == Mode::kSwa3d) {
+            static_assert(kSplit == 2, "the 3-D window mask gives each half one t-slice");
+            if (tok_row && j < seq.nvid) {
+              const RasterGeom& g = p.rg;
+              const int kt = j / p.tile_blocks;
+              const int sb = j - kt * p.tile_blocks;
+              const int kid = seq.ids[kt];
+              const int ktw = kid % g.NW, kth = (kid / g.NW) % g.NH, ktt = kid / (g.NW * g.NH);
+              const uint64_t km = swa3d_half_mask(ktt * g.ct + sb * 2 + half, kth * g.ch,
+                                                  ktw * g.cw, tws, twe);
+  #pragma unroll
+              for (int c = 0; c < kCols; ++c)
+                if (!((km >> c) & 1ull)) s[c] = -INFINITY;
+            }
           }
-        }
+        };
+        load_scores();
+        // exp2(s * sl2 - ref) two at a time, packed to bf16 as they come
+        // (most pairs on the ex2 unit, a fixed share on the FMA pipe); with
+        // kMax the raw maximum is taken on the way
+        uint32_t pk[kCols / 2];
+        auto exp_pack = [&](float ref, auto with_max, float& mx) {
+          const float2 sl2v = make_float2(sl2, sl2);
+          const float neg = (ref == -INFINITY) ? 0.f : -ref;
+          const float2 npv = make_float2(neg, neg);
+          float2 ls = make_float2(0.f, 0.f);
+          float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < kCols; c += 2) {
+            if constexpr (decltype(with_max)::value) {
+              if ((c & 2) == 0) m0 = fmax3(m0, s[c], s[c + 1]);
+              else m1 = fmax3(m1, s[c], s[c + 1]);
+            }
+            const float2 x = __ffma2_rn(make_float2(s[c], s[c + 1]), sl2v, npv);
+            float2 e;
+            if (exp2_on_fma(c / 2)) {   // resolved at compile time (unrolled)
+              e = exp2_fma2(x);
+            } else {
+              e = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            }
+            ls = __fadd2_rn(ls, e);
+            pk[c / 2] = pack_bf16x2(e.x, e.y);
+          }
+          if constexpr (decltype(with_max)::value) mx = fmaxf(m0, m1);
+          return ls.x + ls.y;
+        };
         // row max: four independent chains of three-input max
-        constexpr int kQ = kCols / 4;
-        float mq[4];
+        auto own_max = [&]() {
+          constexpr int kQ = kCols / 4;
+          float mq[4];
 #pragma unroll
-        for (int k4 = 0; k4 < 4; ++k4) {
-          float m = s[k4 * kQ];
+          for (int k4 = 0; k4 < 4; ++k4) {
+            float m = s[k4 * kQ];
 #pragma unroll
-          for (int i = 1; i + 1 < kQ; i += 2) m = fmax3(m, s[k4 * kQ + i], s[k4 * kQ + i + 1]);
-          if constexpr (kQ % 2 == 0) m = fmaxf(m, s[k4 * kQ + kQ - 1]);
-          mq[k4] = m;
-        }
-        float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
-        // The two halves of a row must agree on the reference of the
-        // exponent.  Each half posts its max and goes on with a provisional
-        // reference (the running max, or its own max when that escalates past
-        // the running max by more than 2^8); the partner's max is read only
-        // after the exponentials, and the rare half whose reference was too
-        // low rescales its 64 values.  The exchange latency thus overlaps the
-        // exp2 work instead of sitting in front of it.
+            for (int i = 1; i + 1 < kQ; i += 2) m = fmax3(m, s[k4 * kQ + i], s[k4 * kQ + i + 1]);
+            if constexpr (kQ % 2 == 0) m = fmaxf(m, s[k4 * kQ + kQ - 1]);
+            mq[k4] = m;
+          }
+          return fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+        };
+        // the halves of a row agree on the block's max through shared memory
         float* rb = red + ((j & 1) * 2 + slot) * 2 * kBM;
-        if constexpr (kSplit == 2) {
-          rb[half * kBM + r] = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xb);
-        }
-        const float m_loc = mx * sl2;
-        const float m_prov = m_loc > m_run + 8.0f ? m_loc : m_run;
-        const float neg_p = (m_prov == -INFINITY) ? 0.f : -m_prov;
-        // exp2 of the scaled, shifted scores, in place
-        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-        for (int c = 0; c < kCols; c += 2) {
-          s[c] = fast_exp2(fmaf(s[c], sl2, neg_p));
-          s[c + 1] = fast_exp2(fmaf(s[c + 1], sl2, neg_p));
-          ls0 += s[c];
-          ls1 += s[c + 1];
-        }
-        if constexpr (kSplit == 2) {
-          if (!mbar_wait_warp(xb, j & 1, abort_flag)) { done = false; break; }
-          mx = fmaxf(mx, rb[(half ^ 1) * kBM + r]);
-        }
-        const float m_cand = mx * sl2;
-        const bool resc = m_cand > m_run + 8.0f;
+        auto exchange_max = [&](float& mx) {
+          if constexpr (kSplit == 2) {
+            rb[half * kBM + r] = mx;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(xb);
+            if (!mbar_wait_warp(xb, j & 1, abort_flag)) return false;
+            mx = fmaxf(mx, rb[(half ^ 1) * kBM + r]);
+          }
+          return true;
+        };
+        // Reference of the exponent: the running max (log2 units), raised
+        // only when the block's max exceeds it by more than 2^8.  Rows that
+        // have a running max take the exponentials against it at once and
+        // the block's max on the way; in the rare case that max raises the
+        // reference, the block is recomputed from its scores in TMEM.  A warp
+        // with a row that has no running max yet (its first unmasked block)
+        // agrees on the max first.  Both halves of a row see the same rows'
+        // state, so they take the same branches.
+        using kNoMax = std::integral_constant<bool, false>;
+        using kWithMax = std::integral_constant<bool, true>;
+        float mx = -INFINITY;
+        float lsum;
+        bool resc;
         float alpha = 1.f;
-        if (resc) {
-          alpha = fast_exp2(m_run - m_cand);
-          m_run = m_cand;
-          l_run *= alpha;
-        }
-        if (m_run > m_prov) {
-          const float corr = fast_exp2(m_prov - m_run);
-#pragma unroll
-          for (int c = 0; c < kCols; ++c) s[c] *= corr;
-          ls0 *= corr;
-          ls1 *= corr;
+        if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
+          mx = own_max();
+          if (!exchange_max(mx)) { done = false; break; }
+          const float m_cand = mx * sl2;
+          resc = m_cand > m_run + 8.0f;
+          if (resc) {
+            alpha = fast_exp2(m_run - m_cand);
+            m_run = m_cand;
+            l_run *= alpha;
+          }
+          lsum = exp_pack(m_run, kNoMax{}, mx);
+        } else {
+          lsum = exp_pack(m_run, kWithMax{}, mx);
+          if (!exchange_max(mx)) { done = false; break; }
+          const float m_cand = mx * sl2;
+          resc = m_cand > m_run + 8.0f;
+          if (resc) {
+            alpha = fast_exp2(m_run - m_cand);
+            m_run = m_cand;
+            l_run *= alpha;
+          }
+          if (__any_sync(0xffffffffu, resc)) {
+            load_scores();
+            lsum = exp_pack(m_run, kNoMax{}, mx);
+          }
         }
         // bf16 P over the first half of this thread's own score columns
 #pragma unroll
-        for (int cc = 0; cc < kCols / 32; ++cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(s[cc * 32 + 2 * e], s[cc * 32 + 2 * e + 1]);
-          STA_TMEM_ST16(t_p + cc * 16, pk);
-        }
-        l_run += ls0 + ls1;
+        for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_ST16(t_p + cc * 16, (pk + cc * 16));
+        l_run += lsum;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
           for (int cc = 0; cc < kOCols / 32; ++cc) {
