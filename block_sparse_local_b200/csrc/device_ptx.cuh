@@ -484,9 +484,14 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 // Pairs of a softmax's score columns whose exponentials go through
-// exp2_fma2: kExp2FmaPairs of every 8 (3/8 measured best on B200: the ex2
-// unit and the issue slots then finish together).
-constexpr int kExp2FmaPairs = 3;
+// exp2_fma2: kExp2FmaPairs of every 8.  Measured in the forward kernel on
+// B200 (video+text workload): 0 -> 14.58 ms, 1 -> 14.00, 2 -> 13.96,
+// 3 -> 14.15, 4 -> 15.10; in a stand-alone exp loop 3 was best, but the
+// kernel's loop also packs P and takes the row max on the FMA/ALU pipes.
+#ifndef STA_EXP2_FMA_PAIRS
+#define STA_EXP2_FMA_PAIRS 2
+#endif
+constexpr int kExp2FmaPairs = STA_EXP2_FMA_PAIRS;
 __host__ __device__ constexpr bool exp2_on_fma(int pair) {
   return ((pair * kExp2FmaPairs) / 8) != (((pair + 1) * kExp2FmaPairs) / 8);
 }
