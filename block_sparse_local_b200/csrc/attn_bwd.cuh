@@ -22,6 +22,8 @@
 // halves as two K ranges.
 #pragma once
 
+#include <type_traits>
+
 #include "device_ptx.cuh"
 #include "attn_fwd.cuh"
 
@@ -42,8 +44,8 @@ struct BwdParams {
   int text_sentinel;      // lists end with the text block
   float scale_log2;       // log2(e) / sqrt(d)
   float scale;            // 1 / sqrt(d)
-  const float* lse2;      // [rows] log-sum-exp in log2 units
-  const float* delta;     // [rows] D
+  const float* neg_lse2;  // [rows] minus the log-sum-exp in log2 units
+  const float* neg_delta; // [rows] minus D
   __nv_bfloat16* out_a;   // dQ (dQ kernel) or dK (dK/dV kernel)
   __nv_bfloat16* out_b;   // dV (dK/dV kernel)
 };
@@ -63,12 +65,13 @@ struct BwdCfg {
 };
 
 // One warp per two rows: D[row] = sum_c dO[row,c] * O[row,c] (fp32) and the
-// log-sum-exp converted to log2 units.
+// log-sum-exp converted to log2 units, both stored negated (the backward
+// kernels add them: P = exp2(S log2(e)/sqrt(d) + neg_lse2), dP + neg_delta).
 template <int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
     const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ dout,
-    const float* __restrict__ lse, float* __restrict__ delta, float* __restrict__ lse2,
-    long long rows) {
+    const float* __restrict__ lse, float* __restrict__ neg_delta,
+    float* __restrict__ neg_lse2, long long rows) {
   constexpr int kLanes = D / 8;                       // 16-byte vectors per row
   constexpr int kRowsPerWarp = 32 / kLanes;
   const long long warp = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5;
@@ -91,8 +94,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(
 #pragma unroll
   for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (row < rows && lane % kLanes == 0) {
-    delta[row] = acc;
-    lse2[row] = lse[row] * 1.4426950408889634f;
+    neg_delta[row] = -acc;
+    neg_lse2[row] = -lse[row] * 1.4426950408889634f;
   }
 }
 
@@ -219,50 +222,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && !skip) {
+    // A thread's TMA loads complete one after another, so every operand
+    // panel has its own lane: lanes 0 .. kPanels-1 the panels of the first
+    // streamed operand (Q for dK/dV, K for dQ) and of the resident K / Q,
+    // lanes kPanels .. 2 kPanels-1 those of the second (dO / V, resident
+    // V / dO), lane 2 kPanels the two 512-byte LSE / D copies (dK/dV).  Lane
+    // 0 posts the expected bytes of every stage.
+    constexpr int kPanels = C::kPanels;
+    constexpr int kLanes = 2 * kPanels + (kDKV ? 1 : 0);
+    if (lane < kLanes && !skip) {
       const uint64_t pol = policy_evict_last();
       const int row0 = item.q0;   // the resident block
-      mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
-#pragma unroll
-      for (int pn = 0; pn < C::kPanels; ++pn) {
-        tma_load_2d_hint(smem + C::kResA + pn * C::kPanelBytes, kDKV ? &tmap_k : &tmap_q,
-                         res_full, pn * 64, row0, pol);
-        tma_load_2d_hint(smem + C::kResB + pn * C::kPanelBytes, kDKV ? &tmap_v : &tmap_do,
+      const bool is_b = lane >= kPanels && lane < 2 * kPanels;
+      const bool is_vec = lane == 2 * kPanels;
+      const int pn = lane % kPanels;
+      if (lane == 0) mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
+      if (!is_vec) {
+        const CUtensorMap* mres = is_b ? (kDKV ? &tmap_v : &tmap_do) : (kDKV ? &tmap_k : &tmap_q);
+        tma_load_2d_hint(smem + (is_b ? C::kResB : C::kResA) + pn * C::kPanelBytes, mres,
                          res_full, pn * 64, row0, pol);
       }
-      int issued = 0;
+      const CUtensorMap* mstr = is_b ? (kDKV ? &tmap_do : &tmap_v) : (kDKV ? &tmap_q : &tmap_k);
       for (int j = 0; j < n; ++j) {
         const int st = j % ST;
         if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
         const int row = stream_row(j);
         uint8_t* base = smem + C::kStream + st * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + (kDKV ? 1024 : 0));
-#pragma unroll
-        for (int pn = 0; pn < C::kPanels; ++pn) {
-          tma_load_2d_hint(base + pn * C::kPanelBytes, kDKV ? &tmap_q : &tmap_k, &full[st],
-                           pn * 64, row, pol);
-          tma_load_2d_hint(base + C::kBlockBytes + pn * C::kPanelBytes,
-                           kDKV ? &tmap_do : &tmap_v, &full[st], pn * 64, row, pol);
-        }
-        if constexpr (kDKV) {
-          // the streamed query block's lse2 and D (2 x 512 bytes)
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + (kDKV ? 1024 : 0));
+        if (!is_vec) {
+          tma_load_2d_hint(base + (is_b ? C::kBlockBytes : 0) + pn * C::kPanelBytes, mstr,
+                           &full[st], pn * 64, row, pol);
+        } else if constexpr (kDKV) {
+          // the streamed query block's -lse2 and -D (2 x 512 bytes)
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
               "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes)),
-              "l"(reinterpret_cast<uint64_t>(p.lse2 + row)), "r"(smem_u32(&full[st]))
+              "l"(reinterpret_cast<uint64_t>(p.neg_lse2 + row)), "r"(smem_u32(&full[st]))
               : "memory");
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
               "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes + 512)),
-              "l"(reinterpret_cast<uint64_t>(p.delta + row)), "r"(smem_u32(&full[st]))
+              "l"(reinterpret_cast<uint64_t>(p.neg_delta + row)), "r"(smem_u32(&full[st]))
               : "memory");
         }
-        issued = j + 1;
       }
-      mbar_wait_drain(res_full, 0);
-      for (int s = 0; s < ST && s < issued; ++s) {
-        const int last = s + ((issued - 1 - s) / ST) * ST;
-        mbar_wait_drain(&full[s], (last / ST) & 1);
+      __syncwarp((1u << kLanes) - 1u);
+      // Leave no copy in flight: wait for the last load of every stage.
+      if (lane == 0) {
+        mbar_wait_drain(res_full, 0);
+        for (int st = 0; st < ST && st < n; ++st) {
+          const int last = st + ((n - 1 - st) / ST) * ST;
+          mbar_wait_drain(&full[st], (last / ST) & 1);
+        }
       }
     }
   } else if (warp == 1) {
@@ -327,15 +338,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint32_t t_s = tmem + lane_off + half * 64;           // S / S^T columns
       const uint32_t t_dp = tmem + lane_off + 128 + half * 64;    // dP / dP^T columns
       const float sl2 = p.scale_log2;
-      // dQ: this query row's lse2 and D; dK/dV: whether this key row is valid
-      float row_lse2 = 0.f, row_delta = 0.f;
+      // dQ: this query row's -lse2 and -D; dK/dV: whether this key row is valid
+      float row_nl2 = 0.f, row_nd = 0.f;
       bool row_valid = true;
       if constexpr (kDKV) {
         const int off = my_row - item.kv_base;
         if (off >= p.L_v) row_valid = (off - p.L_v) < p.text_len;
       } else {
-        row_lse2 = p.lse2[my_row];
-        row_delta = p.delta[my_row];
+        row_nl2 = p.neg_lse2[my_row];
+        row_nd = p.neg_delta[my_row];
       }
       bool done = true;
       for (int j = 0; j < n; ++j) {
@@ -349,7 +360,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         STA_TMEM_LD32(t_dp, (dr + 0));
         STA_TMEM_LD32(t_dp + 32, (dr + 32));
         tmem_wait_ld();
-        // column mask: dQ over the text key block (keys >= text_len)
+        // masks: dQ over the text key block (keys >= text_len, the same for
+        // every row of the block), dK/dV on padded text key rows
         int hi = 64;
         if constexpr (!kDKV) {
           if (j >= nvid) {
@@ -357,32 +369,57 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             hi = p.text_len - col0;
           }
         }
-        const float* vec = reinterpret_cast<const float*>(
-            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes);
+        const bool masked = kDKV ? !__all_sync(0xffffffffu, row_valid) : hi < 64;
+        // dK/dV: -lse2 and -D of the streamed rows, 16-byte aligned in the stage
+        const float4* nl4p = reinterpret_cast<const float4*>(
+            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + half * 16;
+        const float4* nd4p = nl4p + 32;
         uint32_t pk_p[32], pk_ds[32];
+        // P = exp2(S sl2 - lse2) and dS = P (dP - D), two columns at a time
+        // (packed f32x2 FMA / ADD / MUL; a fixed share of the exponentials on
+        // the FMA pipe), packed to bf16 as they come
+        auto elementwise = [&](auto with_mask) {
+          const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int c = 2 * e + u;
-            const float s = __uint_as_float(sr[c]);
-            const float dp = __uint_as_float(dr[c]);
-            float lse2, dl;
+          for (int e4 = 0; e4 < 16; ++e4) {
+            float4 nl4, nd4;
             if constexpr (kDKV) {
-              lse2 = vec[half * 64 + c];
-              dl = vec[128 + half * 64 + c];
+              nl4 = nl4p[e4];
+              nd4 = nd4p[e4];
             } else {
-              lse2 = row_lse2;
-              dl = row_delta;
+              nl4 = make_float4(row_nl2, row_nl2, row_nl2, row_nl2);
+              nd4 = make_float4(row_nd, row_nd, row_nd, row_nd);
             }
-            float pr = fast_exp2(fmaf(s, sl2, -lse2));
-            if (!row_valid || c >= hi) pr = 0.f;
-            pv[u] = pr;
-            dsv[u] = pr * (dp - dl);
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 2 * e4 + h2;       // column pair
+              const int c = 2 * e;
+              const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+              const float2 x = __ffma2_rn(
+                  make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, nl);
+              float2 pr;
+              if (exp2_on_fma(e)) {   // resolved at compile time (unrolled)
+                pr = exp2_fma2(x);
+              } else {
+                pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              }
+              if constexpr (decltype(with_mask)::value) {
+                if (!row_valid || c >= hi) pr.x = 0.f;
+                if (!row_valid || c + 1 >= hi) pr.y = 0.f;
+              }
+              const float2 ds = __fmul2_rn(
+                  pr, __fadd2_rn(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
+                                 nd));
+              pk_p[e] = pack_bf16x2(pr.x, pr.y);
+              pk_ds[e] = pack_bf16x2(ds.x, ds.y);
+            }
           }
-          pk_p[e] = pack_bf16x2(pv[0], pv[1]);
-          pk_ds[e] = pack_bf16x2(dsv[0], dsv[1]);
+        };
+        if (masked) {
+          elementwise(std::true_type{});
+        } else {
+          elementwise(std::false_type{});
         }
         if constexpr (kDKV) {
           STA_TMEM_ST32(t_s, pk_p);     // P^T over the first 32 of this warp's columns

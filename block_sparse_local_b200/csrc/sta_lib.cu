@@ -1062,7 +1062,7 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
   const int NQ = g.NV + (g.has_text ? 1 : 0);
   const int max_k = g.NV + 1;   // both list kinds fit in NV + 1 entries
   const int bpt = g.V / 128;
-  // workspace: lse2, delta, forward lists, transposed lists, two plans
+  // workspace: -lse2, -D, forward lists, transposed lists, two plans
   const size_t vb = align_up(sizeof(float) * size_t(rows), 256);
   const size_t cb = align_up(sizeof(int) * size_t(cls.nclass) * NQ, 256);
   const size_t ib = align_up(sizeof(int) * size_t(cls.nclass) * NQ * max_k, 256);
@@ -1078,8 +1078,8 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
     ws.cap = total;
   }
   uint8_t* w = static_cast<uint8_t*>(ws.buf);
-  float* lse2 = reinterpret_cast<float*>(w);
-  float* delta = reinterpret_cast<float*>(w + vb);
+  float* neg_lse2 = reinterpret_cast<float*>(w);
+  float* neg_delta = reinterpret_cast<float*>(w + vb);
   int* fc = reinterpret_cast<int*>(w + 2 * vb);
   int* tc = reinterpret_cast<int*>(w + 2 * vb + cb);
   int* fi = reinterpret_cast<int*>(w + 2 * vb + 2 * cb);
@@ -1134,17 +1134,17 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
                                cudaMemcpyHostToDevice, st));
   STA_CUDA_TRY(cudaMemcpyAsync(kitems, kv.data(), sizeof(WorkItem) * kv.size(),
                                cudaMemcpyHostToDevice, st));
-  // D and lse2
+  // -D and -lse2
   const long long warps = (rows * (d / 8) + 31) / 32;
   const int pre_blocks = static_cast<int>((warps * 32 + 255) / 256);
   if (d == 128)
     sta::bwd_preprocess_kernel<128><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-        delta, lse2, rows);
+        neg_delta, neg_lse2, rows);
   else
     sta::bwd_preprocess_kernel<64><<<pre_blocks, 256, 0, st>>>(
         static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse,
-        delta, lse2, rows);
+        neg_delta, neg_lse2, rows);
   // forward and transposed tile lists
   launch_lists(fc, fi, cls, g, max_k, st);
   {
@@ -1174,8 +1174,8 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
   prm.text_len = g.text_len;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
   prm.scale = static_cast<float>(1.0 / std::sqrt(double(d)));
-  prm.lse2 = lse2;
-  prm.delta = delta;
+  prm.neg_lse2 = neg_lse2;
+  prm.neg_delta = neg_delta;
   // dQ: forward lists, text key blocks with valid keys
   prm.items = qitems;
   prm.counts = fc;
