@@ -8,18 +8,24 @@
 //
 // Two kernels share one template, one 128-row block per CTA:
 //  * kDKV = false (dQ): resident Q, dO; streams the query block's key
-//    blocks (the forward's tile lists).  TMEM: S [0,128), dP [128,256),
-//    dQ accumulator [256, 256+d).
+//    blocks (the forward's tile lists).  TMEM: dQ accumulator [0, d).
 //  * kDKV = true (dK, dV): resident K, V of one key block; streams the query
 //    blocks whose windows hold that key tile (transposed tile lists), with
-//    their log2-domain LSE and D.  TMEM: S^T [0,128), dP^T [128,256),
-//    dV [256,256+d), dK [256+d, 256+2d).
-// Warps: 0 TMA producer, 1 MMA issuer (S and dP by SS tcgen05.mma, then the
-// accumulators by TS tcgen05.mma with P / dS from TMEM), 2-9 elementwise:
-// two warps per TMEM lane quarter, 64 columns each.  A warp writes its packed
-// bf16 P / dS into the first 32 of its own 64 columns, so no warp overwrites
+//    their log2-domain LSE and D.  TMEM: dV [0, d), dK [d, 2d).
+// Each streamed 128-row block is worked on as two 64-row units, alternating
+// between two TMEM score buffers at columns 256 and 384 (S or S^T in 64
+// columns, dP or dP^T in the next 64), so the tensor cores compute the next
+// unit's scores while the elementwise warps turn this unit's scores into P
+// and dS: with one 128-row buffer (the accumulators leave room for no more
+// at d = 128) the score MMAs, the elementwise work and the accumulate MMAs
+// ran strictly one after another.
+// Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (S and dP
+// by SS tcgen05.mma with N = 64, then the accumulators by TS tcgen05.mma with
+// P / dS from TMEM, K = 64), 2-9 elementwise: two warps per TMEM lane
+// quarter, 32 of the unit's 64 columns each.  A warp writes its packed bf16
+// P / dS into the first 16 of its own 32 columns, so no warp overwrites
 // scores another warp still has to read; the accumulate MMAs take the two
-// halves as two K ranges.
+// column groups as two K ranges.
 #pragma once
 
 #include <type_traits>
@@ -131,12 +137,18 @@ __global__ void __launch_bounds__(128) kv_tile_list_transposed_kernel(
   for (int i = n; i < g.max_k; ++i) out[i] = -1;
 }
 
-// D = A B^T over d (SS, both K-major, 128 x 128 scores).  a, b: descriptors
-// of the two 128-row blocks (address field already offset).
+// TMEM columns: the accumulators (dV at 0 and dK at d, or dQ at 0), then two
+// score buffers of one 64-row unit each: S (or S^T) in 64 columns, dP (or
+// dP^T) in the next 64.
+constexpr uint32_t kBwdBufCol = 256;
+
+// Scores of one 64-row unit of a streamed block: D = A B^T over d (SS, both
+// K-major, M = 128 resident rows, N = 64).  a: resident block descriptor, b:
+// descriptor of the unit's first row (address field already offset).
 template <int D>
-__device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint64_t a, uint64_t b) {
+__device__ __forceinline__ void bwd_issue_ss_unit(uint32_t d_tmem, uint64_t a, uint64_t b) {
   using C = BwdCfg<D>;
-  constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
+  constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
@@ -144,14 +156,17 @@ __device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint64_t a, uint64
   }
 }
 
-// acc (+)= A B with A packed bf16 in TMEM columns [a, a+32) and [a+64, a+96)
-// (K = 128 rows of the streamed block) and B an MN-major block (N = d).
+// acc (+)= A B over one 64-row unit: A packed bf16 in TMEM, K = 64 rows of
+// the unit, columns [a, a+16) (rows 0..31, first column group) and
+// [a+32, a+48) (rows 32..63, second group); B the unit's rows of a streamed
+// block as an MN-major operand (N = d).  ACC: accumulate flag of the first
+// k-step.
 template <int D, bool ACC>
-__device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
+__device__ __forceinline__ void bwd_issue_ts_unit(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
   constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t acol = (kk < 4) ? kk * 8 : 64 + (kk - 4) * 8;
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t acol = (kk >> 1) * 32 + (kk & 1) * 8;
     umma_ts(d_tmem, a_tmem + acol, b + ((kk * 16 * 128) >> 4), kIdAcc, (ACC || kk > 0) ? 1u : 0u);
   }
 }
@@ -171,9 +186,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* res_full = bars;
   uint64_t* full = res_full + 1;         // [ST]
   uint64_t* empty = full + ST;           // [ST]
-  uint64_t* s_full = empty + ST;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* acc_full = p_full + 1;
+  uint64_t* s_full = empty + ST;         // [2] per score buffer
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* acc_full = p_full + 2;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -197,8 +212,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     mbar_init(res_full, 1);
     for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 8);
+    }
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
@@ -286,41 +303,66 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t d_res_b = sdesc_sw128(warp_uniform(s_res_b), 16, 1024);
       const uint64_t d_str_k = sdesc_sw128(warp_uniform(s_stream), 16, 1024);
       const uint64_t d_str_mn = sdesc_sw128(warp_uniform(s_stream), C::kPanelBytes, 1024);
-      bool ok = mbar_wait_warp(res_full, 0, abort_flag);
-      for (int j = 0; ok && j < n; ++j) {
-        const int st = j % ST;
-        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t sa = (static_cast<uint32_t>(st) * C::kStageBytes) >> 4;
-        const uint32_t sb = sa + (C::kBlockBytes >> 4);
+      // Units u = 0 .. 2n-1: the two 64-row halves of streamed block u / 2,
+      // in score buffer u % 2.  Scores of unit u + 2 go into the buffer that
+      // the accumulate MMAs of unit u read, issued right after them (tcgen05
+      // MMAs of one thread execute in issue order), so the scores of the next
+      // unit are computed while the elementwise warps work on this one.
+      const int U = 2 * n;
+      auto issue_scores = [&](int u) {
+        const int st = (u >> 1) % ST;
+        const uint32_t so = (static_cast<uint32_t>(st) * C::kStageBytes + (u & 1) * 64 * 128) >> 4;
+        const uint32_t sb = so + (C::kBlockBytes >> 4);
+        const uint32_t buf = tm + kBwdBufCol + (u & 1) * 128;
         if (elect_one()) {
-          bwd_issue_ss<D>(tm + 0, d_res_a, d_str_k + sa);     // S^T = K Q^T  |  S = Q K^T
-          bwd_issue_ss<D>(tm + 128, d_res_b, d_str_k + sb);   // dP^T = V dO^T |  dP = dO V^T
-          umma_commit(s_full);
+          bwd_issue_ss_unit<D>(buf, d_res_a, d_str_k + so);        // S^T = K Q^T  |  S = Q K^T
+          bwd_issue_ss_unit<D>(buf + 64, d_res_b, d_str_k + sb);   // dP^T = V dO^T |  dP = dO V^T
+          umma_commit(&s_full[u & 1]);
         }
         __syncwarp();
-        if (!mbar_wait_warp(p_full, j & 1, abort_flag)) break;
+      };
+      bool ok = mbar_wait_warp(res_full, 0, abort_flag) && mbar_wait_warp(&full[0], 0, abort_flag);
+      if (ok) {
         tc_fence_after();
+        issue_scores(0);
+        issue_scores(1);
+      }
+      for (int u = 0; ok && u < U; ++u) {
+        const int st = (u >> 1) % ST;
+        if (!mbar_wait_warp(&p_full[u & 1], (u >> 1) & 1, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t so = (static_cast<uint32_t>(st) * C::kStageBytes + (u & 1) * 64 * 128) >> 4;
+        const uint32_t sb = so + (C::kBlockBytes >> 4);
+        const uint32_t buf = tm + kBwdBufCol + (u & 1) * 128;
         if (elect_one()) {
-          if (j > 0) {
+          if (u > 0) {
             if constexpr (kDKV) {
-              bwd_issue_ts<D, true>(tm + 256, tm + 0, d_str_mn + sb);       // dV += P^T dO
-              bwd_issue_ts<D, true>(tm + 256 + D, tm + 128, d_str_mn + sa); // dK += dS^T Q
+              bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + sb);           // dV += P^T dO
+              bwd_issue_ts_unit<D, true>(tm + D, buf + 64, d_str_mn + so);  // dK += dS^T Q
             } else {
-              bwd_issue_ts<D, true>(tm + 256, tm + 0, d_str_mn + sa);       // dQ += dS K
+              bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + so);           // dQ += dS K
             }
           } else {
             if constexpr (kDKV) {
-              bwd_issue_ts<D, false>(tm + 256, tm + 0, d_str_mn + sb);
-              bwd_issue_ts<D, false>(tm + 256 + D, tm + 128, d_str_mn + sa);
+              bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + sb);
+              bwd_issue_ts_unit<D, false>(tm + D, buf + 64, d_str_mn + so);
             } else {
-              bwd_issue_ts<D, false>(tm + 256, tm + 0, d_str_mn + sa);
+              bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + so);
             }
           }
-          umma_commit(&empty[st]);
-          if (j == n - 1) umma_commit(acc_full);
+          if (u & 1) umma_commit(&empty[st]);   // both units of the stage consumed
+          if (u == U - 1) umma_commit(acc_full);
         }
         __syncwarp();
+        const int un = u + 2;
+        if (un < U) {
+          if ((un & 1) == 0) {
+            const int jn = un >> 1;
+            if (!mbar_wait_warp(&full[jn % ST], (jn / ST) & 1, abort_flag)) break;
+            tc_fence_after();
+          }
+          issue_scores(un);
+        }
       }
       if (elect_one()) umma_commit(mma_done);
       __syncwarp();
@@ -335,8 +377,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int my_row = item.q0 + r;
     if (!skip) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + half * 64;           // S / S^T columns
-      const uint32_t t_dp = tmem + lane_off + 128 + half * 64;    // dP / dP^T columns
       const float sl2 = p.scale_log2;
       // dQ: this query row's -lse2 and -D; dK/dV: whether this key row is valid
       float row_nl2 = 0.f, row_nd = 0.f;
@@ -349,39 +389,44 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         row_nd = p.neg_delta[my_row];
       }
       bool done = true;
-      for (int j = 0; j < n; ++j) {
+      for (int u = 0; u < 2 * n; ++u) {
+        const int j = u >> 1;           // streamed block
+        const int hu = u & 1;           // its 64-row half, and the score buffer
         const int st = j % ST;
-        if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
-        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
+        if (!mbar_wait_warp(&s_full[hu], j & 1, abort_flag)) { done = false; break; }
+        if constexpr (kDKV) {
+          if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
+        }
         tc_fence_after();
-        uint32_t sr[64], dr[64];
-        STA_TMEM_LD32(t_s, (sr + 0));
-        STA_TMEM_LD32(t_s + 32, (sr + 32));
-        STA_TMEM_LD32(t_dp, (dr + 0));
-        STA_TMEM_LD32(t_dp + 32, (dr + 32));
+        const uint32_t t_s = tmem + lane_off + kBwdBufCol + hu * 128 + half * 32;
+        const uint32_t t_dp = t_s + 64;
+        uint32_t sr[32], dr[32];
+        STA_TMEM_LD32(t_s, sr);
+        STA_TMEM_LD32(t_dp, dr);
         tmem_wait_ld();
         // masks: dQ over the text key block (keys >= text_len, the same for
         // every row of the block), dK/dV on padded text key rows
-        int hi = 64;
+        int hi = 32;
         if constexpr (!kDKV) {
           if (j >= nvid) {
-            const int col0 = (j - nvid) * 128 + half * 64;
+            const int col0 = (j - nvid) * 128 + hu * 64 + half * 32;
             hi = p.text_len - col0;
           }
         }
-        const bool masked = kDKV ? !__all_sync(0xffffffffu, row_valid) : hi < 64;
-        // dK/dV: -lse2 and -D of the streamed rows, 16-byte aligned in the stage
+        const bool masked = kDKV ? !__all_sync(0xffffffffu, row_valid) : hi < 32;
+        // dK/dV: -lse2 and -D of this warp's 32 streamed rows, 16-byte
+        // aligned in the stage
         const float4* nl4p = reinterpret_cast<const float4*>(
-            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + half * 16;
+            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + hu * 16 + half * 8;
         const float4* nd4p = nl4p + 32;
-        uint32_t pk_p[32], pk_ds[32];
+        uint32_t pk_p[16], pk_ds[16];
         // P = exp2(S sl2 - lse2) and dS = P (dP - D), two columns at a time
         // (packed f32x2 FMA / ADD / MUL; a fixed share of the exponentials on
         // the FMA pipe), packed to bf16 as they come
         auto elementwise = [&](auto with_mask) {
           const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
+          for (int e4 = 0; e4 < 8; ++e4) {
             float4 nl4, nd4;
             if constexpr (kDKV) {
               nl4 = nl4p[e4];
@@ -421,16 +466,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         } else {
           elementwise(std::false_type{});
         }
+        // packed bf16 over the first 16 of this warp's own 32 columns, so no
+        // warp overwrites scores another warp still has to read
         if constexpr (kDKV) {
-          STA_TMEM_ST32(t_s, pk_p);     // P^T over the first 32 of this warp's columns
-          STA_TMEM_ST32(t_dp, pk_ds);   // dS^T likewise in the dP^T columns
+          STA_TMEM_ST16(t_s, pk_p);     // P^T
+          STA_TMEM_ST16(t_dp, pk_ds);   // dS^T
         } else {
-          STA_TMEM_ST32(t_s, pk_ds);    // dS over the S columns
+          STA_TMEM_ST16(t_s, pk_ds);    // dS over the S columns
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(p_full);
+        if (lane == 0) mbar_arrive(&p_full[hu]);
       }
       if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
         tc_fence_after();
@@ -438,8 +485,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int nacc = kDKV ? 2 : 1;
         for (int a = 0; a < nacc; ++a) {
           // dK/dV kernel: a = 0 -> dV (unscaled), a = 1 -> dK (scaled)
-          const uint32_t t_acc = tmem + lane_off + 256 + (kDKV && a == 0 ? 0 : (kDKV ? D : 0)) +
-                                 half * kHalfCols;
+          const uint32_t t_acc = tmem + lane_off + (kDKV && a == 1 ? D : 0) + half * kHalfCols;
           const float sc = (kDKV && a == 0) ? 1.f : p.scale;
           __nv_bfloat16* dstp = (kDKV && a == 0) ? p.out_b : p.out_a;
           uint4* dst = reinterpret_cast<uint4*>(dstp + static_cast<size_t>(my_row) * D +
