@@ -2,14 +2,14 @@
 
 README "Sliding Tile Atteniton Kernel", section Usage:
   * the video is a (T, H, W) token grid, flattened in raster order;
-  * "a tile is a cube of size (6, 8, 8)";
-  * "window_size in tiles": window (3,3,3) lets a query attend to
+  * tiles are (6, 8, 8) blocks of tokens (t, h, w);
+  * the window is given in tiles: window (3,3,3) lets a query attend to
     (3x6, 3x8, 3x8) = (18, 24, 24) tokens, i.e. a window counts whole tiles
     and every query sees a full window;
   * 256 text tokens (with padding) follow the video tokens;
     ``text_length`` ranges over 0..256.
 
-Readings taken where the page is silent (each is listed in the design doc):
+Readings taken where the page is silent:
   * the window is centred on the query tile, start = c - floor(w/2), and
     shifted inward at the grid border so that it always spans w tiles
     (pinned for odd windows by the hand-derived fixtures; for an even window
@@ -19,7 +19,7 @@ Readings taken where the page is silent (each is listed in the design doc):
   * with has_text=False there are no text rows at all.
 """
 
-TEXT_PAD = 256  # README Usage: "text tokens = 256 with padding"
+TEXT_PAD = 256  # README Usage: the text block is padded to 256 tokens
 
 
 def tile_grid(T, H, W, tile):

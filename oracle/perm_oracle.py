@@ -2,8 +2,8 @@
 
 TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
 
-README "Sliding Tile Atteniton Kernel", Usage: "a tile is a cube of size
-(6, 8, 8)".  A tile's tokens have to be contiguous rows of q, k, v for the
+README "Sliding Tile Atteniton Kernel", Usage: tiles are (6, 8, 8) blocks of
+tokens.  A tile's tokens have to be contiguous rows of q, k, v for the
 tile-by-tile blocks of the attention map to be dense ("Why is STA Fast?").
 Reading (the page does not fix the order): tiles in tile-major raster order,
 tokens inside a tile in raster order, text rows left in place.

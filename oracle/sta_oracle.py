@@ -16,9 +16,9 @@ followed by the padded text block of 256 rows):
   3. text query (i >= L_v): allowed iff j is a video key, or a text key with
      u < text_len.  (Padded text query rows u >= text_len follow the same
      rule as valid text rows.)
-Rules 2 and 3 are the reading taken for the text tokens the README's Usage
-section appends ("If your attention contains text token"); the page gives no
-formula for them.
+Rules 2 and 3 are the reading taken for the optional text tokens that the
+README's Usage section appends after the video; the page gives no formula for
+them.
 
 Two independent forms are provided and cross-checked by the tests:
   * form A: an explicit S x S boolean mask and a masked softmax (tiny only);

@@ -2,9 +2,10 @@
 
 TEST INFRASTRUCTURE ONLY (see oracle/__init__.py).
 
-README "Sliding Tile Atteniton Kernel", Usage ("window_size in tiles") and
-"Why is STA Fast?" ("STA removes mixed blocks"): a query tile attends to
-whole key tiles, so the work of one query tile is a list of key tiles.
+README "Sliding Tile Atteniton Kernel", Usage (the window is counted in
+tiles) and "Why is STA Fast?" (STA has no partially masked blocks): a query
+tile attends to whole key tiles, so the work of one query tile is a list of
+key tiles.
 
 Encoding (the library's bit-exact contract):
   * tiles are numbered in tile-major raster order,
