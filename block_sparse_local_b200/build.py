@@ -15,7 +15,8 @@ LIB_PATH = os.path.join(HERE, "libsta.so")
 SOURCES = [os.path.join(HERE, "csrc", "sta_lib.cu")]
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
                      ("device_ptx.cuh", "reorder.cuh", "tile_lists.cuh",
-                      "attn_fwd.cuh", "attn_fwd_pair.cuh", "attn_bwd.cuh", "hilbert.cuh")] + [os.path.join(ROOT, "include", "sta.h")]
+                      "attn_fwd.cuh", "attn_fwd_pair.cuh", "attn_bwd.cuh", "attn_bwd_dq.cuh",
+                      "hilbert.cuh")] + [os.path.join(ROOT, "include", "sta.h")]
 
 
 def nvcc_path():

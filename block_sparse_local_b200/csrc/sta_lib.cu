@@ -24,6 +24,7 @@
 #include "attn_fwd_pair.cuh"
 #include "hilbert.cuh"
 #include "attn_bwd.cuh"
+#include "attn_bwd_dq.cuh"
 
 namespace {
 
@@ -1013,16 +1014,26 @@ template <int D, bool kDKV>
 sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mdo, const sta::BwdParams& prm, int num_items,
                       cudaStream_t st) {
-  constexpr int smem = sta::BwdCfg<D>::kSmemBytes;
+  // dK/dV: attn_bwd_kernel (64-row units); dQ: attn_bwd_dq_kernel (K and V
+  // in separate rings, next block's scores during this block's elementwise work)
+  constexpr int smem = kDKV ? sta::BwdCfg<D>::kSmemBytes : sta::BwdDqCfg<D>::kSmemBytes;
   static bool attr_set[64] = {};
   int dev = 0;
   STA_CUDA_TRY(cudaGetDevice(&dev));
   if (!attr_set[dev]) {
-    STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_kernel<D, kDKV>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    if constexpr (kDKV) {
+      STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_kernel<D, true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    } else {
+      STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_dq_kernel<D>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    }
     attr_set[dev] = true;
   }
-  sta::attn_bwd_kernel<D, kDKV><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+  if constexpr (kDKV)
+    sta::attn_bwd_kernel<D, true><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+  else
+    sta::attn_bwd_dq_kernel<D><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
