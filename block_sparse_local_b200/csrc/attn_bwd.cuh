@@ -6,12 +6,11 @@
 // D_i = sum_c dO_ic O_ic:  dP = dO V^T,  dS = P (dP - D),
 // dQ = dS K / sqrt(d),  dK = dS^T Q / sqrt(d),  dV = P^T dO.
 //
-// Two kernels share one template, one 128-row block per CTA:
-//  * kDKV = false (dQ): resident Q, dO; streams the query block's key
-//    blocks (the forward's tile lists).  TMEM: dQ accumulator [0, d).
-//  * kDKV = true (dK, dV): resident K, V of one key block; streams the query
-//    blocks whose windows hold that key tile (transposed tile lists), with
-//    their log2-domain LSE and D.  TMEM: dV [0, d), dK [d, 2d).
+// This file: the preprocessing (D and the log2-domain LSE), the transposed
+// tile lists, and the dK/dV kernel, one 128-row key block per CTA: resident
+// K, V; streams the query blocks whose windows hold that key tile
+// (transposed tile lists), with their -LSE2 and -D.  TMEM: dV [0, d),
+// dK [d, 2d).  The dQ kernel is in attn_bwd_dq.cuh.
 // Each streamed 128-row block is worked on as two 64-row units, alternating
 // between two TMEM score buffers at columns 256 and 384 (S or S^T in 64
 // columns, dP or dP^T in the next 64), so the tensor cores compute the next
@@ -171,9 +170,9 @@ __device__ __forceinline__ void bwd_issue_ts_unit(uint32_t d_tmem, uint32_t a_tm
   }
 }
 
-template <int D, bool kDKV>
+template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    attn_bwd_kernel(const __grid_constant__ CUtensorMap tmap_q,
+    attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
@@ -246,7 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // V / dO), lane 2 kPanels the two 512-byte LSE / D copies (dK/dV).  Lane
     // 0 posts the expected bytes of every stage.
     constexpr int kPanels = C::kPanels;
-    constexpr int kLanes = 2 * kPanels + (kDKV ? 1 : 0);
+    constexpr int kLanes = 2 * kPanels + 1;
     if (lane < kLanes && !skip) {
       const uint64_t pol = policy_evict_last();
       const int row0 = item.q0;   // the resident block
@@ -255,21 +254,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int pn = lane % kPanels;
       if (lane == 0) mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
       if (!is_vec) {
-        const CUtensorMap* mres = is_b ? (kDKV ? &tmap_v : &tmap_do) : (kDKV ? &tmap_k : &tmap_q);
+        const CUtensorMap* mres = is_b ? &tmap_v : &tmap_k;
         tma_load_2d_hint(smem + (is_b ? C::kResB : C::kResA) + pn * C::kPanelBytes, mres,
                          res_full, pn * 64, row0, pol);
       }
-      const CUtensorMap* mstr = is_b ? (kDKV ? &tmap_do : &tmap_v) : (kDKV ? &tmap_q : &tmap_k);
+      const CUtensorMap* mstr = is_b ? &tmap_do : &tmap_q;
       for (int j = 0; j < n; ++j) {
         const int st = j % ST;
         if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
         const int row = stream_row(j);
         uint8_t* base = smem + C::kStream + st * C::kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + (kDKV ? 1024 : 0));
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + 1024);
         if (!is_vec) {
           tma_load_2d_hint(base + (is_b ? C::kBlockBytes : 0) + pn * C::kPanelBytes, mstr,
                            &full[st], pn * 64, row, pol);
-        } else if constexpr (kDKV) {
+        } else {
           // the streamed query block's -lse2 and -D (2 x 512 bytes)
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
@@ -336,19 +335,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t buf = tm + kBwdBufCol + (u & 1) * 128;
         if (elect_one()) {
           if (u > 0) {
-            if constexpr (kDKV) {
-              bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + sb);           // dV += P^T dO
-              bwd_issue_ts_unit<D, true>(tm + D, buf + 64, d_str_mn + so);  // dK += dS^T Q
-            } else {
-              bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + so);           // dQ += dS K
-            }
+            bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + sb);           // dV += P^T dO
+            bwd_issue_ts_unit<D, true>(tm + D, buf + 64, d_str_mn + so);  // dK += dS^T Q
           } else {
-            if constexpr (kDKV) {
-              bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + sb);
-              bwd_issue_ts_unit<D, false>(tm + D, buf + 64, d_str_mn + so);
-            } else {
-              bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + so);
-            }
+            bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + sb);
+            bwd_issue_ts_unit<D, false>(tm + D, buf + 64, d_str_mn + so);
           }
           if (u & 1) umma_commit(&empty[st]);   // both units of the stage consumed
           if (u == U - 1) umma_commit(acc_full);
@@ -378,15 +369,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (!skip) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
       const float sl2 = p.scale_log2;
-      // dQ: this query row's -lse2 and -D; dK/dV: whether this key row is valid
-      float row_nl2 = 0.f, row_nd = 0.f;
+      // whether this key row is valid (padded text keys are not)
       bool row_valid = true;
-      if constexpr (kDKV) {
+      {
         const int off = my_row - item.kv_base;
         if (off >= p.L_v) row_valid = (off - p.L_v) < p.text_len;
-      } else {
-        row_nl2 = p.neg_lse2[my_row];
-        row_nd = p.neg_delta[my_row];
       }
       bool done = true;
       for (int u = 0; u < 2 * n; ++u) {
@@ -394,9 +381,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int hu = u & 1;           // its 64-row half, and the score buffer
         const int st = j % ST;
         if (!mbar_wait_warp(&s_full[hu], j & 1, abort_flag)) { done = false; break; }
-        if constexpr (kDKV) {
-          if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
-        }
+        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
         const uint32_t t_s = tmem + lane_off + kBwdBufCol + hu * 128 + half * 32;
         const uint32_t t_dp = t_s + 64;
@@ -404,18 +389,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         STA_TMEM_LD32(t_s, sr);
         STA_TMEM_LD32(t_dp, dr);
         tmem_wait_ld();
-        // masks: dQ over the text key block (keys >= text_len, the same for
-        // every row of the block), dK/dV on padded text key rows
-        int hi = 32;
-        if constexpr (!kDKV) {
-          if (j >= nvid) {
-            const int col0 = (j - nvid) * 128 + hu * 64 + half * 32;
-            hi = p.text_len - col0;
-          }
-        }
-        const bool masked = kDKV ? !__all_sync(0xffffffffu, row_valid) : hi < 32;
-        // dK/dV: -lse2 and -D of this warp's 32 streamed rows, 16-byte
-        // aligned in the stage
+        // padded text key rows give zero P and dS
+        const bool masked = !__all_sync(0xffffffffu, row_valid);
+        // -lse2 and -D of this warp's 32 streamed rows, 16-byte aligned in
+        // the stage
         const float4* nl4p = reinterpret_cast<const float4*>(
             smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + hu * 16 + half * 8;
         const float4* nd4p = nl4p + 32;
@@ -427,14 +404,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const float2 sl2v = make_float2(sl2, sl2);
 #pragma unroll
           for (int e4 = 0; e4 < 8; ++e4) {
-            float4 nl4, nd4;
-            if constexpr (kDKV) {
-              nl4 = nl4p[e4];
-              nd4 = nd4p[e4];
-            } else {
-              nl4 = make_float4(row_nl2, row_nl2, row_nl2, row_nl2);
-              nd4 = make_float4(row_nd, row_nd, row_nd, row_nd);
-            }
+            const float4 nl4 = nl4p[e4];
+            const float4 nd4 = nd4p[e4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int e = 2 * e4 + h2;       // column pair
@@ -450,8 +421,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
               }
               if constexpr (decltype(with_mask)::value) {
-                if (!row_valid || c >= hi) pr.x = 0.f;
-                if (!row_valid || c + 1 >= hi) pr.y = 0.f;
+                if (!row_valid) pr = make_float2(0.f, 0.f);
               }
               const float2 ds = __fmul2_rn(
                   pr, __fadd2_rn(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
@@ -468,12 +438,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         // packed bf16 over the first 16 of this warp's own 32 columns, so no
         // warp overwrites scores another warp still has to read
-        if constexpr (kDKV) {
-          STA_TMEM_ST16(t_s, pk_p);     // P^T
-          STA_TMEM_ST16(t_dp, pk_ds);   // dS^T
-        } else {
-          STA_TMEM_ST16(t_s, pk_ds);    // dS over the S columns
-        }
+        STA_TMEM_ST16(t_s, pk_p);     // P^T
+        STA_TMEM_ST16(t_dp, pk_ds);   // dS^T
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -482,12 +448,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
         tc_fence_after();
         constexpr int kHalfCols = D / 2;
-        const int nacc = kDKV ? 2 : 1;
-        for (int a = 0; a < nacc; ++a) {
-          // dK/dV kernel: a = 0 -> dV (unscaled), a = 1 -> dK (scaled)
-          const uint32_t t_acc = tmem + lane_off + (kDKV && a == 1 ? D : 0) + half * kHalfCols;
-          const float sc = (kDKV && a == 0) ? 1.f : p.scale;
-          __nv_bfloat16* dstp = (kDKV && a == 0) ? p.out_b : p.out_a;
+        for (int a = 0; a < 2; ++a) {
+          // a = 0 -> dV (unscaled), a = 1 -> dK (scaled)
+          const uint32_t t_acc = tmem + lane_off + (a == 1 ? D : 0) + half * kHalfCols;
+          const float sc = a == 0 ? 1.f : p.scale;
+          __nv_bfloat16* dstp = a == 0 ? p.out_b : p.out_a;
           uint4* dst = reinterpret_cast<uint4*>(dstp + static_cast<size_t>(my_row) * D +
                                                 half * kHalfCols);
 #pragma unroll

@@ -1014,7 +1014,7 @@ template <int D, bool kDKV>
 sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mdo, const sta::BwdParams& prm, int num_items,
                       cudaStream_t st) {
-  // dK/dV: attn_bwd_kernel (64-row units); dQ: attn_bwd_dq_kernel (K and V
+  // dK/dV: attn_bwd_dkv_kernel (64-row units); dQ: attn_bwd_dq_kernel (K and V
   // in separate rings, next block's scores during this block's elementwise work)
   constexpr int smem = kDKV ? sta::BwdCfg<D>::kSmemBytes : sta::BwdDqCfg<D>::kSmemBytes;
   static bool attr_set[64] = {};
@@ -1022,7 +1022,7 @@ sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
   STA_CUDA_TRY(cudaGetDevice(&dev));
   if (!attr_set[dev]) {
     if constexpr (kDKV) {
-      STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_kernel<D, true>,
+      STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_dkv_kernel<D>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
     } else {
       STA_CUDA_TRY(cudaFuncSetAttribute(sta::attn_bwd_dq_kernel<D>,
@@ -1031,7 +1031,7 @@ sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     attr_set[dev] = true;
   }
   if constexpr (kDKV)
-    sta::attn_bwd_kernel<D, true><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    sta::attn_bwd_dkv_kernel<D><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
   else
     sta::attn_bwd_dq_kernel<D><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
   STA_CUDA_TRY(cudaGetLastError());
