@@ -62,6 +62,8 @@ def parse():
     ap.add_argument("--no-swa", action="store_true", help="skip the SWA comparison")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with fewer heads (profiling captures only)")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the backward pass of the workload (profiling captures)")
     return ap.parse_args()
 
 
@@ -94,6 +96,29 @@ def attn_traffic(units_per_launch):
         return None
     # captured on a smaller case; traffic scales with the key blocks processed
     return d["dram_bytes_per_unit"] * units_per_launch
+
+
+def run_backward(q, k, v, w, shape, pairs, dev, stream):
+    """Backward pass of the STA workload (tile order): dQ, dK, dV from the
+    saved LSE; algorithmic work 5 matmuls of 2*d per retained pair."""
+    qt, kt, vt = (sta.tile_reorder(x, shape, w.tile, w.has_text) for x in (q, k, v))
+    ot, lset = sta.forward(qt, kt, vt, w.windows, w.text_len, w.has_text, shape, w.tile,
+                           return_lse=True)
+    dot = torch.randn_like(qt, dtype=torch.float32).to(torch.bfloat16)
+    for _ in range(2):
+        sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape, w.tile)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(3):
+        sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape, w.tile)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    bms = a.elapsed_time(b) / 3
+    sta.device_status(dev)
+    return {"workload": w.name, "ms": bms,
+            "effective_tflops": 10.0 * w.d * pairs / (bms * 1e-3) / 1e12,
+            "flop_model": "10*d per retained pair (5 matmuls)"}
 
 
 class ClockSampler:
@@ -266,6 +291,13 @@ def run_ours(args):
     pairs = sta.retained_pairs(w.B, w.windows, shape, w.tile, w.text_len, w.has_text)
     flops = 4.0 * w.d * pairs
 
+    if args.backward_only:
+        if rank == 0:
+            print(json.dumps({"backward_only": run_backward(q, k, v, w, shape, pairs, dev,
+                                                            stream)}))
+        if world > 1:
+            dist.destroy_process_group()
+        return
     attn_ev = []
 
     def step(record=False):
@@ -441,28 +473,8 @@ def run_ours(args):
         swa["hilbert_slide2d"] = hil
         del hq, hk, hv, ho
 
-        # backward pass of the same STA workload (tile order): dQ, dK, dV from
-        # the saved LSE; algorithmic work 5 matmuls of 2*d per retained pair
-        qt, kt, vt = (sta.tile_reorder(x, shape, w.tile, w.has_text) for x in (q, k, v))
-        ot, lset = sta.forward(qt, kt, vt, w.windows, w.text_len, w.has_text, shape, w.tile,
-                               return_lse=True)
-        dot = torch.randn_like(qt, dtype=torch.float32).to(torch.bfloat16)
-        for _ in range(2):
-            sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape,
-                         w.tile)
-        torch.cuda.synchronize(dev)
-        a.record(stream)
-        for _ in range(3):
-            sta.backward(qt, kt, vt, ot, dot, lset, w.windows, w.text_len, w.has_text, shape,
-                         w.tile)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        bms = a.elapsed_time(b) / 3
-        sta.device_status(dev)
-        swa["backward"] = {"workload": w.name, "ms": bms,
-                           "effective_tflops": 10.0 * w.d * pairs / (bms * 1e-3) / 1e12,
-                           "flop_model": "10*d per retained pair (5 matmuls)"}
-        del qt, kt, vt, ot, lset, dot
+        # backward pass of the same STA workload
+        swa["backward"] = run_backward(q, k, v, w, shape, pairs, dev, stream)
 
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
