@@ -101,6 +101,8 @@ def attn_traffic(units_per_launch):
 def run_backward(q, k, v, w, shape, pairs, dev, stream):
     """Backward pass of the STA workload (tile order): dQ, dK, dV from the
     saved LSE; algorithmic work 5 matmuls of 2*d per retained pair."""
+    import torch
+    import block_sparse_local_b200 as sta
     qt, kt, vt = (sta.tile_reorder(x, shape, w.tile, w.has_text) for x in (q, k, v))
     ot, lset = sta.forward(qt, kt, vt, w.windows, w.text_len, w.has_text, shape, w.tile,
                            return_lse=True)
