@@ -1137,7 +1137,15 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
     return a.first > b.first;
   };
   std::stable_sort(qp.begin(), qp.end(), by_len);
-  std::stable_sort(kp.begin(), kp.end(), by_len);
+  // dK/dV: stream lengths differ from key tile to key tile (border tiles lie
+  // in more windows), so a global longest-first order would interleave the
+  // (batch, head) slices and the CTAs running at once would stream every
+  // slice's Q and dO through L2; keep slices together, longest first inside
+  auto by_slice_len = [](const std::pair<int, WorkItem>& a, const std::pair<int, WorkItem>& b) {
+    if (a.second.kv_base != b.second.kv_base) return a.second.kv_base < b.second.kv_base;
+    return a.first > b.first;
+  };
+  std::stable_sort(kp.begin(), kp.end(), by_slice_len);
   std::vector<WorkItem> qv, kv;
   for (auto& e : qp) qv.push_back(e.second);
   for (auto& e : kp) kv.push_back(e.second);
