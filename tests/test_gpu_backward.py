@@ -44,6 +44,10 @@ CASES = [
     ((6, 8, 16), (6, 8, 8), [(1, 1, 2)], 200, True, 64),
     ((4, 8, 16), (2, 8, 8), [(2, 1, 2)], 256, True, 128),
     ((4, 8, 16), (2, 8, 8), [(1, 1, 1)], 0, True, 64),    # text rows, no valid text key
+    # 2 and 3 key blocks per video query block: fewer than the dQ kernel's
+    # three K stages, so its rings and drains run partly empty
+    ((2, 8, 16), (2, 8, 8), [(1, 1, 1)], 100, True, 128),
+    ((2, 8, 16), (2, 8, 8), [(1, 1, 2)], 100, True, 128),
 ]
 
 
