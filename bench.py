@@ -77,10 +77,16 @@ def load_peaks():
 
 
 def source_hash():
+    """Hash of the attention kernel's code (comment-only lines and blank lines
+    left out, so that editing a comment keeps the measured traffic valid)."""
     h = hashlib.sha256()
     for rel in ATTN_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            for line in f:
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(t.encode())
+                    h.update(b"\n")
     return h.hexdigest()[:16]
 
 

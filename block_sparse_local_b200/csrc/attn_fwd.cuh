@@ -16,8 +16,9 @@
 //
 // CTA = 2 + 8 * kSplit warps (18 with kSplit = 2), one work item = up to
 // two 128-row query blocks ("slots") that read the same key blocks:
-//   warp 0      TMA producer (one thread): Q once, then K and V blocks into
-//               K / V rings of shared-memory stages (128-byte swizzle).
+//   warp 0      TMA producer, one lane per operand panel: Q once, then K
+//               and V blocks into K / V rings of shared-memory stages
+//               (128-byte swizzle).
 //   warp 1      MMA issuer (the whole warp waits, one elected lane issues)
 //               and TMEM owner: S_i = Q_i K^T (SS, M=128 N=128 K=d),
 //               O_i += P_i V (TS: P from TMEM, V from shared memory, N=d),
@@ -25,10 +26,12 @@
 //               slot while the other slot's softmax runs.
 //   warps 2..   softmax, 4 * kSplit warps per slot: kSplit warps share each
 //               query row (TMEM lane), each with 128 / kSplit of its scores;
-//               they update the running max / sum, write bf16 P over the
-//               first half of their own score columns, rescale their O
-//               columns when the max grew by more than 2^8, and finally
-//               normalise O and store it.
+//               exponentials two at a time with packed f32x2 arithmetic (a
+//               share of them on the FMA pipe) against the running max, the
+//               block max taken in the same loop; they update the running
+//               max / sum, write bf16 P over the first half of their own
+//               score columns, rescale their O columns when the max grew by
+//               more than 2^8, and finally normalise O and store it.
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 // O1 [256+d, 256+2d); P_i aliases half of S_i.  The MMA that overwrites S_i
 // with the next scores is issued after the P_i.V MMA that reads P_i;
