@@ -1,6 +1,6 @@
 // reorder.cuh - raster <-> tile token permutation (bit-exact row copies).
 //
-// STA README, Usage: "a tile is a cube of size (6, 8, 8)".  For the
+// STA README, Usage: tiles are (6, 8, 8) blocks of tokens.  For the
 // tile-by-tile blocks of the attention map to be dense ("Why is STA Fast?")
 // the tokens of one tile must be contiguous rows.  Video row
 // r = (t*H + h)*W + w lives at tile-ordered row tile_id*V + in_tile with

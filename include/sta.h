@@ -4,11 +4,11 @@
  * Method: the STA README ("Sliding Tile Atteniton Kernel", FastVideo
  * sta_kernel/thunderkitten), sections "Usage", "How Does STA Work?" and
  * "Why is STA Fast?".  A (T,H,W) video token grid is cut into tiles of
- * (ct,ch,cw) tokens ("a tile is a cube of size (6, 8, 8)"); every query tile
- * attends to the whole key tiles inside a window of (wt,wh,ww) tiles
- * ("window_size in tiles"), centred on the query tile and shifted inward at
- * the grid border so it always spans the full window; 256 padded text tokens
- * may follow the video ("text tokens = 256 with padding", text_length 0..256).
+ * (ct,ch,cw) tokens (the page's tiles are (6, 8, 8)); every query tile
+ * attends to the whole key tiles inside a window of (wt,wh,ww) tiles (the
+ * window is counted in tiles), centred on the query tile and shifted inward at
+ * the grid border so it always spans the full window; a text block padded to
+ * 256 tokens may follow the video (text_length 0..256).
  * Video queries also attend to the first text_len text keys; text queries
  * attend to every video key and the first text_len text keys.  The attention
  * map is therefore made of fully dense or fully empty tile blocks.
@@ -50,7 +50,7 @@ typedef enum sta_status {
                                  STA_NOALLOC_SCRATCH_BYTES of scratch            */
 } sta_status;
 
-/* Text block size (README Usage: "text tokens = 256 with padding"). */
+/* Text block size (README Usage: the text block is padded to 256 tokens). */
 #define STA_TEXT_PAD 256
 
 /*
@@ -197,7 +197,7 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v,
 /*
  * sta_swa3d_forward - token-level 3-D sliding-window attention, the
  * mixed-block baseline that README "Why is STA Fast?" compares STA with
- * ("2D/3D Sliding Window Attention (SWA) creates many mixed blocks").  Every
+ * (token-level windows leave many partially masked blocks).  Every
  * video query token attends to the keys of a window of
  * window_tokens = (Wt, Wh, Ww) TOKENS centred on it and shifted inward at the
  * grid border (clipped to the grid), plus the first text_len text keys; text
