@@ -1140,8 +1140,13 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
   // dK/dV: stream lengths differ from key tile to key tile (border tiles lie
   // in more windows), so a global longest-first order would interleave the
   // (batch, head) slices and the CTAs running at once would stream every
-  // slice's Q and dO through L2; keep slices together, longest first inside
-  auto by_slice_len = [](const std::pair<int, WorkItem>& a, const std::pair<int, WorkItem>& b) {
+  // slice's Q and dO through L2.  The text key blocks (every query block of
+  // their slice, the longest items by far) go first, so that none of them
+  // starts near the end; then the video key blocks slice by slice, longest
+  // first inside a slice.
+  auto by_slice_len = [&](const std::pair<int, WorkItem>& a, const std::pair<int, WorkItem>& b) {
+    const bool ta = a.second.list % NQ == g.NV, tb = b.second.list % NQ == g.NV;
+    if (ta != tb) return ta;
     if (a.second.kv_base != b.second.kv_base) return a.second.kv_base < b.second.kv_base;
     return a.first > b.first;
   };
