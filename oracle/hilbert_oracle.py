@@ -84,16 +84,6 @@ def block_classes(n, window, order, block=128):
     return cls
 
 
-def block_lists(n, window, order, block=128):
-    """Per query block: ascending non-empty key blocks and their class (1/2)."""
-    cls = block_classes(n, window, order, block)
-    lists = []
-    for qb in range(cls.shape[0]):
-        kbs = np.nonzero(cls[qb])[0]
-        lists.append((kbs, cls[qb, kbs]))
-    return lists
-
-
 def block_rectangles(n, order, block=128):
     """(x0, x1, y0, y1) inclusive bounds of every block, asserting that each
     block is a full rectangle (true for Hilbert blocks of 2 * 4^k tokens and

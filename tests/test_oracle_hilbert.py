@@ -1,10 +1,74 @@
 """Pins of the Hilbert-order oracle: the curve's defining properties and the
 block statistics of 2-D slide attention."""
+import os
+
 import numpy as np
 import pytest
 
 from oracle import hilbert_oracle as ho
 from oracle import swa3d_oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def test_curve_n4_equals_hand_derived_sequence():
+    # tests/golden/hilbert_n4.txt: the 16 cells derived by hand from the
+    # 2 x 2 curve and the quadrant rotations (a wrong sub-quadrant
+    # orientation that stays continuous changes this sequence)
+    want = []
+    with open(os.path.join(GOLDEN, "hilbert_n4.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                d, x, y = (int(t) for t in line.split())
+                assert d == len(want)
+                want.append((x, y))
+    assert [ho.hilbert_d2xy(4, d) for d in range(16)] == want
+
+
+@pytest.mark.parametrize("n", [4, 8, 16, 32])
+def test_every_level_is_the_curve_of_its_quadrant(n):
+    # Recursive structure at every level s: positions [m s^2, (m+1) s^2) fill
+    # one aligned s x s square, and the curve inside it, moved to the origin,
+    # is the s x s curve itself, one of its two diagonal reflections, or its
+    # half turn (the composition of both reflections, which appears from the
+    # third level on).
+    order = ho.hilbert_order(n)
+    xs, ys = order % n, order // n
+    s = 2
+    while s <= n:
+        base = [ho.hilbert_d2xy(s, d) for d in range(s * s)]
+        transposed = [(y, x) for x, y in base]
+        anti = [(s - 1 - y, s - 1 - x) for x, y in base]
+        for m in range(n * n // (s * s)):
+            cx, cy = xs[m * s * s:(m + 1) * s * s], ys[m * s * s:(m + 1) * s * s]
+            x0, y0 = cx.min(), cy.min()
+            assert x0 % s == 0 and y0 % s == 0
+            assert cx.max() - x0 == s - 1 and cy.max() - y0 == s - 1
+            local = list(zip((cx - x0).tolist(), (cy - y0).tolist()))
+            mirrored = [(s - 1 - x, s - 1 - y) for x, y in base]
+            assert local in (base, transposed, anti, mirrored), (s, m)
+        s *= 2
+
+
+def test_block_classes_equal_a_plain_loop():
+    # every (query, key) pair tested one by one from its (x, y) coordinates,
+    # small blocks so that partial, full and empty blocks all occur
+    n, w, block = 8, 3, 8
+    for order in (ho.raster_order(n), ho.hilbert_order(n)):
+        nb = n * n // block
+        cnt = np.zeros((nb, nb), dtype=np.int64)
+        for i in range(n * n):
+            qx, qy = int(order[i]) % n, int(order[i]) // n
+            x_lo = min(max(qx - w // 2, 0), n - w)
+            y_lo = min(max(qy - w // 2, 0), n - w)
+            for j in range(n * n):
+                kx, ky = int(order[j]) % n, int(order[j]) // n
+                if x_lo <= kx < x_lo + w and y_lo <= ky < y_lo + w:
+                    cnt[i // block, j // block] += 1
+        want = np.where(cnt == 0, 0, np.where(cnt == block * block, 2, 1))
+        got = ho.block_classes(n, w, order, block)
+        assert np.array_equal(got, want)
+        assert (got == 1).any() and (got == 0).any()
 
 
 @pytest.mark.parametrize("n", [2, 4, 8, 16, 64])
