@@ -66,29 +66,48 @@ def sta_backward_query_rows(q, k, v, dout, rows, T, H, W, tile, window, text_len
     return dq
 
 
+def _query_groups(T, H, W, tile, has_text):
+    """Query rows grouped by the key set they share: the raster rows of each
+    video query tile, then (with text) the 256 text rows."""
+    N = sta_oracle.tile_grid(T, H, W, tile)
+    groups = []
+    for t in range(N[0]):
+        for h in range(N[1]):
+            for w in range(N[2]):
+                groups.append(np.sort(sta_oracle._box_rows(T, H, W, tile, (t, h, w),
+                                                           (1, 1, 1))))
+    if has_text:
+        Lv = T * H * W
+        groups.append(np.arange(Lv, Lv + sta_oracle.TEXT_PAD))
+    return groups
+
+
 def sta_backward_key_rows(q, k, v, dout, keys_wanted, T, H, W, tile, window, text_len,
                           has_text):
-    """dK, dV of the given key rows: every query that attends to one of them
-    is found by scanning the allowed-key sets of all query rows."""
+    """dK, dV of the given key rows (one (batch, head), raster order).
+
+    Every query row whose allowed set holds a wanted key contributes; rows of
+    one query tile (and the text rows) share their allowed set, so each such
+    group is one gather: S, P, O, dP and dS of the group's rows over its
+    allowed keys, then the wanted keys' columns of P^T dO and dS^T q."""
     S, d = q.shape
     scale = 1.0 / np.sqrt(d)
-    want = {int(j): pos for pos, j in enumerate(keys_wanted)}
-    dk = np.zeros((len(keys_wanted), d))
-    dv = np.zeros((len(keys_wanted), d))
-    # query rows whose allowed set meets the wanted keys (tiles share sets)
-    for r in range(S):
-        keys = sta_oracle.allowed_keys(r, T, H, W, tile, window, text_len, has_text)
-        hit = [j for j in keys_wanted if j in set(keys.tolist())] if len(want) < 8 else \
-            np.intersect1d(keys, np.asarray(keys_wanted)).tolist()
-        if not hit:
+    wanted = np.asarray(keys_wanted, dtype=np.int64)
+    dk = np.zeros((len(wanted), d))
+    dv = np.zeros((len(wanted), d))
+    for rows in _query_groups(T, H, W, tile, has_text):
+        keys = sta_oracle.allowed_keys(int(rows[0]), T, H, W, tile, window, text_len, has_text)
+        hit = np.isin(wanted, keys)
+        if not hit.any():
             continue
-        (_, p, o, _), = _rows_fwd(q, k, v, [r], T, H, W, tile, window, text_len, has_text)
-        dp = v[keys] @ dout[r]
-        delta = dout[r] @ o
+        s = (q[rows] @ k[keys].T) * scale
+        p = np.exp(s - s.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        o = p @ v[keys]
+        dp = dout[rows] @ v[keys].T
+        delta = (dout[rows] * o).sum(axis=1, keepdims=True)
         ds = p * (dp - delta)
-        index = {int(j): c for c, j in enumerate(keys)}
-        for j in hit:
-            c = index[int(j)]
-            dv[want[int(j)]] += p[c] * dout[r]
-            dk[want[int(j)]] += ds[c] * q[r] * scale
+        cols = np.searchsorted(keys, wanted[hit])
+        dv[hit] += p[:, cols].T @ dout[rows]
+        dk[hit] += (ds[:, cols].T @ q[rows]) * scale
     return dk, dv

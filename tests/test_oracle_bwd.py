@@ -75,3 +75,14 @@ def test_row_forms_match_dense():
                                                   text_len, True)
     np.testing.assert_allclose(gk, dk[keys], atol=1e-12)
     np.testing.assert_allclose(gv, dv[keys], atol=1e-12)
+    assert not gk[-1].any() and not gv[-1].any()      # padded text key: no gradient
+    # without text, border and interior key tiles, every key row
+    S = T * H * W
+    q, k, v, do = (x[:S] for x in (q, k, v, do))
+    _, dk, dv, _, _ = sta_bwd_oracle.sta_backward_dense(q, k, v, do, T, H, W, tile, window, 0,
+                                                        False)
+    keys = np.arange(S)
+    gk, gv = sta_bwd_oracle.sta_backward_key_rows(q, k, v, do, keys, T, H, W, tile, window, 0,
+                                                  False)
+    np.testing.assert_allclose(gk, dk, atol=1e-12)
+    np.testing.assert_allclose(gv, dv, atol=1e-12)
