@@ -7,8 +7,13 @@ heads against the float64 oracle, row by row
 (oracle.sta_bwd_oracle.sta_backward_query_rows), with the tolerance of the
 small backward tests (max-abs <= 2e-2 max|ref|, mean-abs <= 1e-2 mean|ref|).
 
-dK, dV: two identities of the gradient, checked for every (batch, head) and
-column; they hold at any size, so they cover every key row:
+dK, dV: sampled key rows of two heads against the float64 oracle, element
+by element (oracle.sta_bwd_oracle.sta_backward_key_rows, same tolerance):
+rows of the text key block (valid and padded keys), of a corner video tile
+(in the windows of the most query tiles once the window is shifted inward)
+and of a mid-grid tile, and random video rows.  Also two identities of the
+gradient, checked for every (batch, head) and column; they hold at any size,
+so they cover every key row:
   sum over key rows of dV = sum over query rows of dO
       (dV = P^T dO and every row of P sums to one);
   sum over key rows of dK = 0
@@ -46,12 +51,23 @@ def full_backward():
                               shape, w.tile)
     sta.device_status()
     dq_raster = sta.tile_unreorder(dq, shape, w.tile, w.has_text)
+    dk_raster = sta.tile_unreorder(dk, shape, w.tile, w.has_text)
+    dv_raster = sta.tile_unreorder(dv, shape, w.tile, w.has_text)
     sta.device_status()
-    return w, (q, k, v, dout), dq_raster, dk, dv
+    return w, (q, k, v, dout), dq_raster, dk, dv, dk_raster, dv_raster
+
+
+def _tile_rows(w, tc, count, rng):
+    """`count` raster rows of the video tile with tile coordinates tc."""
+    ct, ch, cw = w.tile
+    t = tc[0] * ct + rng.integers(0, ct, count)
+    h = tc[1] * ch + rng.integers(0, ch, count)
+    x = tc[2] * cw + rng.integers(0, cw, count)
+    return (t * w.H + h) * w.W + x
 
 
 def test_full_dq_sampled_rows(full_backward):
-    w, (q, k, v, dout), dq, _, _ = full_backward
+    w, (q, k, v, dout), dq = full_backward[:3]
     rng = np.random.default_rng(17)
     rows = np.unique(np.concatenate([rng.integers(0, w.L_v, size=48),
                                      np.arange(w.L_v, w.S, 16)]))
@@ -66,8 +82,29 @@ def test_full_dq_sampled_rows(full_backward):
         assert err.mean() <= 1e-2 * np.abs(ref).mean(), (h, err.mean(), np.abs(ref).mean())
 
 
+def test_full_dk_dv_sampled_key_rows(full_backward):
+    w, (q, k, v, dout), _, _, _, dk, dv = full_backward
+    rng = np.random.default_rng(23)
+    text = w.L_v + np.array([0, 63, 127, 128, 199, 200, 255])   # 200.. are padding
+    keys = np.unique(np.concatenate([text, _tile_rows(w, (0, 0, 0), 12, rng),
+                                     _tile_rows(w, (2, 3, 5), 12, rng),
+                                     rng.integers(0, w.L_v, 12)]))
+    for h in (3, 20):
+        q64, k64, v64, do64 = (x[0, h].double().cpu().numpy() for x in (q, k, v, dout))
+        rk, rv = sta_bwd_oracle.sta_backward_key_rows(q64, k64, v64, do64, keys, w.T, w.H,
+                                                      w.W, w.tile, tuple(w.windows[h]),
+                                                      w.text_len, w.has_text)
+        for name, got_all, ref in (("dk", dk, rk), ("dv", dv, rv)):
+            got = got_all[0, h].float().cpu().numpy()[keys]
+            err = np.abs(got - ref)
+            assert err.max() <= 2e-2 * np.abs(ref).max(), (name, h, err.max())
+            assert err.mean() <= 1e-2 * np.abs(ref).mean(), (name, h, err.mean())
+            pad = keys >= w.L_v + w.text_len
+            assert not got[pad].any(), (name, h)       # padded text keys: exactly zero
+
+
 def test_full_dv_column_sums_equal_dout_column_sums(full_backward):
-    w, (_, _, _, dout), _, _, dv = full_backward
+    w, (_, _, _, dout), _, _, dv = full_backward[:5]
     sdv = dv.double().sum(dim=2)                      # [B, heads, d]
     sdo = dout.double().sum(dim=2)
     scale = dout.double().pow(2).sum(dim=2).sqrt()
@@ -76,7 +113,7 @@ def test_full_dv_column_sums_equal_dout_column_sums(full_backward):
 
 
 def test_full_dk_column_sums_vanish(full_backward):
-    _, _, _, dk, _ = full_backward
+    dk = full_backward[3]
     sdk = dk.double().sum(dim=2)
     scale = dk.double().pow(2).sum(dim=2).sqrt()
     ratio = (sdk.abs() / scale).max().item()

@@ -42,17 +42,22 @@ def test_reorder_bit_exact(B, nh, d, shape, tile, has_text):
 
 
 def test_reorder_full_size_video_text():
+    # every element of two heads carries its own (head, row, column) code, so
+    # the whole output is checked against the oracle's index formula
     w = workloads.VIDEO_TEXT
-    x = torch.arange(w.S, dtype=torch.int32, device="cuda")
-    x = x[None, None, :, None].expand(w.B, 2, w.S, w.d).contiguous()
-    xb = (x % 65536).to(torch.int16).view(torch.bfloat16).contiguous()
+    heads = 2
+    row = torch.arange(w.S, dtype=torch.int32, device="cuda")[None, :, None]
+    col = torch.arange(w.d, dtype=torch.int32, device="cuda")[None, None, :]
+    hd = torch.arange(heads, dtype=torch.int32, device="cuda")[:, None, None]
+    code = (row * 131 + col * 7 + hd * 1009) % 65536 - 32768
+    xb = code.to(torch.int16)[None].contiguous().view(torch.bfloat16)
     y = sta.tile_reorder(xb, (w.T, w.H, w.W), w.tile, True)
     p = perm_oracle.tile_position_of_raster(w.T, w.H, w.W, w.tile)
     inv = np.empty_like(p)
     inv[p] = np.arange(p.size)
-    expect_rows = np.concatenate([inv, np.arange(w.L_v, w.S)]) % 65536
-    got_rows = y.view(torch.int16)[0, 1, :, 5].to(torch.int32).cpu().numpy() % 65536
-    assert np.array_equal(got_rows, expect_rows)
+    src = torch.from_numpy(np.concatenate([inv, np.arange(w.L_v, w.S)])).cuda()
+    want = xb.view(torch.int16).index_select(2, src)
+    assert torch.equal(y.view(torch.int16), want)
     assert torch.equal(sta.tile_unreorder(y, (w.T, w.H, w.W), w.tile, True).view(torch.int16),
                        xb.view(torch.int16))
     sta.device_status()
