@@ -250,6 +250,41 @@ void tile_box(const Geom& g, const int* w, int t, bool token_mode, int st[3], in
   }
 }
 
+// ------------------------------------------------------------------ stream order
+// A library-owned device buffer (workspace) that calls on different streams
+// share: every call that writes it first waits, on the GPU, for the last call
+// that used it when that call came on another stream, and records an event
+// after its own launches.  Calls on one stream are ordered by the stream
+// itself and pay nothing.  A call made while its stream is being captured
+// into a CUDA graph neither waits nor records (event work across a capture
+// boundary is not allowed); such calls are ordered by their own stream only.
+struct StreamOrder {
+  cudaEvent_t ev = nullptr;
+  cudaStream_t last = nullptr;
+  bool used = false;
+};
+
+bool stream_capturing(cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return false;
+  return cs != cudaStreamCaptureStatusNone;
+}
+
+sta_status order_begin(StreamOrder& o, cudaStream_t st) {
+  if (!o.used || o.last == st || stream_capturing(st)) return STA_OK;
+  STA_CUDA_TRY(cudaStreamWaitEvent(st, o.ev, 0));
+  return STA_OK;
+}
+
+sta_status order_end(StreamOrder& o, cudaStream_t st) {
+  if (stream_capturing(st)) return STA_OK;
+  if (o.ev == nullptr) STA_CUDA_TRY(cudaEventCreateWithFlags(&o.ev, cudaEventDisableTiming));
+  STA_CUDA_TRY(cudaEventRecord(o.ev, st));
+  o.last = st;
+  o.used = true;
+  return STA_OK;
+}
+
 // ------------------------------------------------------------------ workspace
 struct Workspace {
   void* buf = nullptr;
@@ -257,6 +292,7 @@ struct Workspace {
   std::string plan_key;     // key of the plan currently resident in `buf`
   std::vector<WorkItem> items;
   std::vector<int> item_off;  // CTA-pair plans: first item of each cluster, + end
+  StreamOrder order;
 };
 Workspace g_ws[64];
 
@@ -565,6 +601,8 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   const size_t off_bytes = sizeof(int) * offs.size();
   s = ensure_workspace(dev, counts_bytes + ids_bytes + items_bytes + off_bytes);
   if (s != STA_OK) return s;
+  s = order_begin(ws.order, st);
+  if (s != STA_OK) return s;
   uint8_t* wbuf = static_cast<uint8_t*>(ws.buf);
   int* d_counts = reinterpret_cast<int*>(wbuf);
   int* d_ids = reinterpret_cast<int*>(wbuf + counts_bytes);
@@ -625,33 +663,41 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
     s = make_row_map(&mk_half, k, total_rows, d, 64);
     if (s != STA_OK) return s;
   }
-  if (raster) {
-    CUtensorMap q5, k5, v5;
-    const int slices = B * heads;
-    s = make_raster_map(&q5, q, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
-    if (s == STA_OK && pair)
-      s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw,
-                          khalf_t ? box_h : box_h / 2, khalf_t ? box_t / 2 : box_t);
-    else if (s == STA_OK)
-      s = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
-    if (s == STA_OK) s = make_raster_map(&v5, v, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
-    if (s != STA_OK) return s;
-    if (pair) return launch_attn_pair<true>(mq, mk_half, mv, prm, num_items, st, &q5, &k5, &v5);
-    if (token_mode) {
+  auto dispatch = [&]() -> sta_status {
+    if (raster) {
+      CUtensorMap q5, k5, v5;
+      const int slices = B * heads;
+      sta_status r = make_raster_map(&q5, q, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+      if (r == STA_OK && pair)
+        r = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw,
+                            khalf_t ? box_h : box_h / 2, khalf_t ? box_t / 2 : box_t);
+      else if (r == STA_OK)
+        r = make_raster_map(&k5, k, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+      if (r == STA_OK)
+        r = make_raster_map(&v5, v, slices, g.S, g.T, g.H, g.W, d, g.cw, box_h, box_t);
+      if (r != STA_OK) return r;
+      if (pair) return launch_attn_pair<true>(mq, mk_half, mv, prm, num_items, st, &q5, &k5, &v5);
+      if (token_mode) {
+        if (d == 128)
+          return launch_attn<128, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5,
+                                                       &v5);
+        return launch_attn<64, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5,
+                                                    &v5);
+      }
       if (d == 128)
-        return launch_attn<128, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5,
-                                                     &v5);
-      return launch_attn<64, Mode::kSwa3d, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
+        return launch_attn<128, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
+      return launch_attn<64, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
     }
-    if (d == 128)
-      return launch_attn<128, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
-    return launch_attn<64, Mode::kSta, true>(mq, mk, mv, prm, num_items, st, &q5, &k5, &v5);
-  }
-  if (token_mode) return STA_ERR_UNSUPPORTED;
-  if (pair) return launch_attn_pair<false>(mq, mk_half, mv, prm, num_items, st, nullptr, nullptr,
-                                           nullptr);
-  if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
-  return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+    if (token_mode) return STA_ERR_UNSUPPORTED;
+    if (pair)
+      return launch_attn_pair<false>(mq, mk_half, mv, prm, num_items, st, nullptr, nullptr,
+                                     nullptr);
+    if (d == 128) return launch_attn<128, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+    return launch_attn<64, Mode::kSta>(mq, mk, mv, prm, num_items, st);
+  };
+  s = dispatch();
+  if (s != STA_OK) return s;
+  return order_end(ws.order, st);
 }
 
 // ------------------------------------------------------------------ host-buffer pipeline
@@ -862,6 +908,9 @@ struct NoAllocState {
   unsigned char* scratch = nullptr;   // device address of g_noalloc_scratch
   std::string plan_key;               // host-side plan cache (host memory only)
   std::vector<WorkItem> items;
+  // Key of the plan whose items are in the device array.  Only this entry
+  // point writes the array, so an unchanged key means the items are there.
+  std::string resident_key;
 };
 NoAllocState g_noalloc[64];
 
@@ -929,9 +978,15 @@ sta_status forward_noalloc_impl(const void* q, const void* k, const void* v, voi
   if (s == STA_OK) s = make_row_map(&mk, k, total_rows, d);
   if (s == STA_OK) s = make_row_map(&mv, v, total_rows, d);
   if (s != STA_OK) return s;
-  // The array keeps the previous call's contents: the plan is rewritten on
-  // every call, and the list kernel rewrites every count and id it reads.
-  STA_CUDA_TRY(cudaMemcpyAsync(d_items, na.items.data(), items_bytes, cudaMemcpyHostToDevice, st));
+  // The array keeps the previous call's contents: the plan is copied in only
+  // when it differs from the one already there, and the list kernel rewrites
+  // every count and id that the attention kernel reads.
+  if (na.resident_key != key) {
+    na.resident_key.clear();
+    STA_CUDA_TRY(cudaMemcpyAsync(d_items, na.items.data(), items_bytes, cudaMemcpyHostToDevice,
+                                 st));
+    na.resident_key = key;
+  }
   launch_lists(d_counts, d_ids, cls, g, max_k, st);
   STA_CUDA_TRY(cudaGetLastError());
 
@@ -963,6 +1018,7 @@ struct Slide2dWs {
   void* buf = nullptr;
   size_t cap = 0;
   std::string key;
+  StreamOrder order;
 };
 Slide2dWs g_ws2d[64];
 
@@ -1007,6 +1063,7 @@ void launch_coords_rects(uint32_t* coords, int4* rects, int n, int order, cudaSt
 struct BwdWs {
   void* buf = nullptr;
   size_t cap = 0;
+  StreamOrder order;
 };
 BwdWs g_wsb[64];
 
@@ -1088,6 +1145,8 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
     STA_CUDA_TRY(cudaMalloc(&ws.buf, total));
     ws.cap = total;
   }
+  s = order_begin(ws.order, st);
+  if (s != STA_OK) return s;
   uint8_t* w = static_cast<uint8_t*>(ws.buf);
   float* neg_lse2 = reinterpret_cast<float*>(w);
   float* neg_delta = reinterpret_cast<float*>(w + vb);
@@ -1219,8 +1278,10 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
   prm.text_blocks = 2;
   prm.out_a = static_cast<__nv_bfloat16*>(dk);
   prm.out_b = static_cast<__nv_bfloat16*>(dv);
-  return d == 128 ? launch_bwd<128, true>(mq, mk, mv, mdo, prm, int(kv.size()), st)
-                  : launch_bwd<64, true>(mq, mk, mv, mdo, prm, int(kv.size()), st);
+  s = d == 128 ? launch_bwd<128, true>(mq, mk, mv, mdo, prm, int(kv.size()), st)
+               : launch_bwd<64, true>(mq, mk, mv, mdo, prm, int(kv.size()), st);
+  if (s != STA_OK) return s;
+  return order_end(ws.order, st);
 }
 
 }  // namespace
@@ -1349,6 +1410,8 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   const size_t bytes = sizeof(WorkItem) * (cached ? ws.items.size() : fresh.size());
   s = ensure_workspace(dev, bytes);
   if (s != STA_OK) return s;
+  s = order_begin(ws.order, st);
+  if (s != STA_OK) return s;
   WorkItem* d_items = static_cast<WorkItem*>(ws.buf);
   if (ws.plan_key != key) {
     ws.items = std::move(fresh);
@@ -1369,8 +1432,10 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   prm.out = static_cast<__nv_bfloat16*>(out);
   prm.lse = nullptr;
   const int num_items = static_cast<int>(ws.items.size());
-  if (d == 128) return launch_attn<128, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
-  return launch_attn<64, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
+  s = d == 128 ? launch_attn<128, Mode::kSwa>(mq, mk, mv, prm, num_items, st)
+               : launch_attn<64, Mode::kSwa>(mq, mk, mv, prm, num_items, st);
+  if (s != STA_OK) return s;
+  return order_end(ws.order, st);
 }
 
 sta_status sta_debug_pair_kernel(int pair) {
@@ -1436,12 +1501,14 @@ sta_status sta_build_slide_block_lists(int* counts, int* ids, int* classes, int 
   uint32_t* coords = reinterpret_cast<uint32_t*>(w);
   int4* rects = reinterpret_cast<int4*>(w + cbytes);
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  s = order_begin(g_ws2d[dev].order, st);
+  if (s != STA_OK) return s;
   launch_coords_rects(coords, rects, n, order, st);
   const size_t smem = sizeof(int) * (512 + nb);
   sta::slide_block_list_kernel<<<nb, 256, smem, st>>>(counts, ids, classes, max_k, coords, rects,
                                                       nb, n, window, 1);
   STA_CUDA_TRY(cudaGetLastError());
-  return STA_OK;
+  return order_end(g_ws2d[dev].order, st);
 }
 
 sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void* out, int B,
@@ -1478,6 +1545,8 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void
   WorkItem* items = reinterpret_cast<WorkItem*>(w + cbytes + rbytes + nbytes + ibytes);
   const std::string key = "s2d:" + std::to_string(B) + ":" + std::to_string(heads) + ":" +
                           std::to_string(n) + ":" + std::to_string(order);
+  s = order_begin(ws.order, st);
+  if (s != STA_OK) return s;
   if (ws.key != key) {
     std::vector<WorkItem> plan;
     plan.reserve(size_t(B) * heads * np);
@@ -1513,8 +1582,10 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
   prm.out = static_cast<__nv_bfloat16*>(out);
   const int num_items = B * heads * np;
-  if (d == 128) return launch_attn<128, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
-  return launch_attn<64, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
+  s = d == 128 ? launch_attn<128, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st)
+               : launch_attn<64, Mode::kSlide2d>(mq, mk, mv, prm, num_items, st);
+  if (s != STA_OK) return s;
+  return order_end(ws.order, st);
 }
 
 sta_status sta_backward(const void* q, const void* k, const void* v, const void* out,
@@ -1551,20 +1622,28 @@ void sta_shutdown(void) {
   std::lock_guard<std::mutex> lock(g_mu);
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return;
+  // cudaFree waits for the device, so no kernel still reads a buffer
+  auto drop_event = [](StreamOrder& o) {
+    if (o.ev != nullptr) cudaEventDestroy(o.ev);
+    o = StreamOrder();
+  };
   for (int i = 0; i < 64; ++i) {
-    if (g_ws[i].buf != nullptr) {
+    if (g_ws[i].buf != nullptr || g_ws[i].order.ev != nullptr) {
       cudaSetDevice(i);
-      cudaFree(g_ws[i].buf);
+      if (g_ws[i].buf != nullptr) cudaFree(g_ws[i].buf);
+      drop_event(g_ws[i].order);
       g_ws[i] = Workspace();
     }
-    if (g_wsb[i].buf != nullptr) {
+    if (g_wsb[i].buf != nullptr || g_wsb[i].order.ev != nullptr) {
       cudaSetDevice(i);
-      cudaFree(g_wsb[i].buf);
+      if (g_wsb[i].buf != nullptr) cudaFree(g_wsb[i].buf);
+      drop_event(g_wsb[i].order);
       g_wsb[i] = BwdWs();
     }
-    if (g_ws2d[i].buf != nullptr) {
+    if (g_ws2d[i].buf != nullptr || g_ws2d[i].order.ev != nullptr) {
       cudaSetDevice(i);
-      cudaFree(g_ws2d[i].buf);
+      if (g_ws2d[i].buf != nullptr) cudaFree(g_ws2d[i].buf);
+      drop_event(g_ws2d[i].order);
       g_ws2d[i] = Slide2dWs();
     }
   }

@@ -25,9 +25,14 @@
  *  - Outputs must not alias inputs.
  *  - Device-side waits are bounded: a kernel that gives up records
  *    STA_ERR_DEVICE_TIMEOUT in a device flag, read by sta_device_status().
- *  - The library keeps one lazily grown device workspace per device (tile
- *    lists and the work plan of sta_forward); calls that use it must not
- *    overlap on different streams.  sta_shutdown() releases it.
+ *  - The library keeps lazily grown device workspaces per device (tile
+ *    lists and work plans of the forward, backward and 2-D entry points).
+ *    A call that writes a workspace first waits, on the GPU, for the last
+ *    call that used it if that call came on another stream (an event per
+ *    workspace), so calls on several streams are ordered in the order the
+ *    host made them; calls on one stream pay nothing for this.  Calls made
+ *    while their stream is being captured into a CUDA graph are ordered by
+ *    that stream only.  sta_shutdown() releases the workspaces.
  */
 #ifndef STA_H_
 #define STA_H_
@@ -91,6 +96,13 @@ sta_status sta_build_kv_tile_lists(int* counts, int* ids, int max_k, int heads,
 
 /*
  * sta_forward - fused STA attention, tile-ordered q,k,v -> out.
+ * Defining passages: README "Usage" (the call
+ * sliding_tile_attention(q, k, v, window_size, text_length, has_text): one
+ * window of tiles per head, text padded to 256 tokens of which text_length
+ * are valid) and "Why is STA Fast?" (a query tile attends to whole key tiles,
+ * so every 128 x 128 block of the attention map is fully dense or fully
+ * empty; only the padded text columns need a mask).  Output row i is
+ * sum_j softmax_j(q_i . k_j / sqrt(d)) v_j over the allowed keys j.
  *   q, k, v: [B, heads, S, d] bf16 device, TILE order (sta_tile_reorder)
  *   out:     [B, heads, S, d] bf16 device, tile order
  *   d in {64, 128}; tile volume ct*ch*cw a multiple of 128;
@@ -98,14 +110,20 @@ sta_status sta_build_kv_tile_lists(int* counts, int* ids, int max_k, int heads,
  *   has_text == 0).  Scale 1/sqrt(d).  bf16 inputs, fp32 accumulation and
  *   softmax, probabilities rounded to bf16 for the P.V product, output
  *   rounded to nearest even.  Runs on sm_100 only (tcgen05 / TMEM / TMA).
+ * Errors: STA_ERR_INVALID_ARG (null or unaligned pointers, aliasing, shape,
+ * window or text_len out of range), STA_ERR_UNSUPPORTED (d, tile volume,
+ * device), STA_ERR_CUDA; all checked before anything is enqueued.
  */
 sta_status sta_forward(const void* q, const void* k, const void* v, void* out,
                        int B, int heads, int d, int T, int H, int W,
                        const int tile[3], const int* window, int text_len,
                        int has_text, void* stream);
 
-/* sta_forward_lse - sta_forward that also writes the natural-log
- * log-sum-exp of every query row to `lse` (device fp32 [B, heads, S]). */
+/* sta_forward_lse - sta_forward (same passages: README "Usage" and "Why is
+ * STA Fast?", same arguments and errors) that also writes the natural-log
+ * log-sum-exp of every query row, ln sum_j exp(q_i . k_j / sqrt(d)) over the
+ * allowed keys, to `lse` (device fp32 [B, heads, S], 4-byte aligned; the
+ * saved statistic of the backward pass). */
 sta_status sta_forward_lse(const void* q, const void* k, const void* v,
                            void* out, float* lse, int B, int heads, int d,
                            int T, int H, int W, const int tile[3],
@@ -305,20 +323,31 @@ int64_t sta_retained_pairs(int B, int heads, int T, int H, int W,
  * latency-bound loop that cannot take the implicit device synchronisation of
  * cudaMalloc / cudaFree.
  *
- * Same arguments, layout, numerics and errors as sta_forward.  The scratch
- * that sta_forward keeps in its lazily grown workspace (KV tile lists and the
- * work plan) lives instead in one file-scope device array of
+ * Same arguments, layout and numerics as sta_forward; it always runs the
+ * one-SM attention kernel (the CTA-pair kernel that sta_debug_pair_kernel(1)
+ * selects for sta_forward is never used here), so its output equals
+ * sta_forward's with the default kernel bit for bit.  The scratch that
+ * sta_forward keeps in its lazily grown workspace (KV tile lists and the work
+ * plan) lives instead in one file-scope device array of
  * STA_NOALLOC_SCRATCH_BYTES, which every GPU that loads libsta.so holds until
- * the process exits.  A problem whose tile lists and plan do not fit returns
- * STA_ERR_SCRATCH_LIMIT before anything is enqueued (the video+text workload
- * of 115,456 tokens x 24 heads needs about 0.55 MiB).
+ * the process exits.
+ *
+ * Errors: those of sta_forward, plus STA_ERR_SCRATCH_LIMIT when the
+ * problem's tile lists and plan do not fit the array (the video+text
+ * workload of 115,456 tokens x 24 heads needs about 0.55 MiB).  That size
+ * check runs on the host after the argument checks and before the device is
+ * queried, so a problem too large for the array gets STA_ERR_SCRATCH_LIMIT
+ * even where sta_forward would answer STA_ERR_UNSUPPORTED for the device.
+ * Nothing is enqueued on any error.
  *
  * The first call on a device looks up that device's address of the array
  * (cudaGetSymbolAddress, with the device current), so make the first call on
  * each device outside any stream capture.  All calls share the one array and
- * it keeps the last call's contents; every call rewrites what it reads, so
- * nothing needs clearing, but calls that overlap on the GPU (different
- * streams, or several host threads) race on it: order them on one stream.
+ * it keeps the last call's contents.  The work plan is copied into it from
+ * host memory only when the problem differs from the previous call's; the
+ * tile lists are rebuilt by a kernel on every call, so nothing needs
+ * clearing.  Calls that overlap on the GPU (different streams, or several
+ * host threads) race on the array: order them on one stream.
  * It calls no cudaMalloc, cudaFree or other allocating routine.
  */
 sta_status sta_forward_noalloc(const void* q, const void* k, const void* v,
