@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-swa", action="store_true", help="skip the SWA comparison")
+    ap.add_argument("--no-other-configs", action="store_true",
+                    help="skip the tiny, video-only and 2-D workloads")
     ap.add_argument("--heads", type=int, default=None,
                     help="run the workload with fewer heads (profiling captures only)")
     ap.add_argument("--backward-only", action="store_true",
@@ -102,6 +104,56 @@ def attn_traffic(units_per_launch):
         return None
     # captured on a smaller case; traffic scales with the key blocks processed
     return d["dram_bytes_per_unit"] * units_per_launch
+
+
+def run_other_configs(dev, stream, peak, flush_bytes=256 << 20, iters=5):
+    """The other STA workloads (tiny, video-only with per-head windows, 2-D
+    at (5,5) and at the grid-covering (16,16) window), each as the bench step
+    runs them: tile lists + the attention kernel on raster-ordered tensors.
+    L2 is flushed (a 256 MB write) before every timed call, and each call is
+    timed alone with CUDA events on the launching stream."""
+    import torch
+    import block_sparse_local_b200 as sta
+    from block_sparse_local_b200 import workloads
+    flush = torch.empty(flush_bytes, dtype=torch.uint8, device=dev)
+    res = {}
+    for w in (workloads.TINY, workloads.VIDEO_ONLY, workloads.IMAGE_2D, workloads.IMAGE_2D_FULL):
+        shape = (w.T, w.H, w.W)
+        q, k, v = workloads.sta_inputs(w, device=dev)
+        out = torch.empty_like(q)
+
+        def call():
+            sta.forward_raster(q, k, v, w.windows, w.text_len, w.has_text, shape, w.tile,
+                               out=out)
+
+        for _ in range(2):
+            call()
+        torch.cuda.synchronize(dev)
+        n = iters if w.B * w.heads > 1 else 20
+        times = []
+        for _ in range(n):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            call()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            times.append(a.elapsed_time(b))
+        sta.device_status(dev)
+        ms = statistics.median(times)
+        pairs = sta.retained_pairs(w.B, w.windows, shape, w.tile, w.text_len, w.has_text)
+        tf = 4.0 * w.d * pairs / (ms * 1e-3) / 1e12
+        res[w.name] = {"B": w.B, "heads": w.heads, "d": w.d, "video": list(shape),
+                       "tile": list(w.tile),
+                       "window": list(w.windows[0]) if len(set(w.windows)) == 1 else
+                       "per head: " + ", ".join(f"{c}x{sum(1 for x in w.windows if x == c)}"
+                                                for c in sorted(set(w.windows))),
+                       "ms": ms, "effective_tflops": tf, "pct_of_bf16_peak": 100.0 * tf / peak,
+                       "kernel": f"attn_fwd_kernel<{w.d},kSta,raster>",
+                       "timing": f"median of {n}, L2 flushed before each call"}
+        del q, k, v, out
+    del flush
+    return res
 
 
 def run_backward(q, k, v, w, shape, pairs, dev, stream):
@@ -322,8 +374,10 @@ def run_ours(args):
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    for _ in range(max(3, args.warmup)):
-        step()
+    nvtx = torch.cuda.nvtx
+    with nvtx.range("bench.warmup"):
+        for _ in range(max(3, args.warmup)):
+            step()
     sta.device_status(dev)
     barrier()
     clocks = ClockSampler(local)
@@ -331,14 +385,16 @@ def run_ours(args):
     barrier()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    for _ in range(args.steps):
-        step(record=True)
+    with nvtx.range("bench.timed_steps"):
+        for _ in range(args.steps):
+            step(record=True)
     t1.record(stream)
     barrier()
     clk = clocks.stop()
     sta.device_status(dev)
     ms = t0.elapsed_time(t1) / args.steps
     attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    attn_ms_median = statistics.median(a.elapsed_time(b) for a, b in attn_ev)
     ms, attn_ms = max_over_ranks([ms, attn_ms], device=dev)
     value = world * flops / (ms * 1e-3) / 1e12
 
@@ -361,8 +417,9 @@ def run_ours(args):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         n_e2e = max(3, min(args.steps, 10))
         e0.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
+        with nvtx.range("bench.e2e_steps"):
+            for _ in range(n_e2e):
+                e2e_step()
         e1.record(stream)
         barrier()
         e2e_ms = e0.elapsed_time(e1) / n_e2e
@@ -501,6 +558,11 @@ def run_ours(args):
         # backward pass of the same STA workload
         swa["backward"] = run_backward(q, k, v, w, shape, pairs, dev, stream)
 
+    others = None
+    if rank == 0 and not args.no_other_configs:
+        peaks_o, _ = load_peaks()
+        others = run_other_configs(dev, stream, float(peaks_o["bf16_tflops"]))
+
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (attn_ms * 1e-3) / 1e12
@@ -510,7 +572,7 @@ def run_ours(args):
                 "frac": achieved / peak, "traffic": attn_traffic(units),
                 "kernel": "attn_fwd_kernel<128,kSta,raster>",
                 "peak_source": peak_src + " burst bf16",
-                "attn_ms": attn_ms}
+                "attn_ms": attn_ms, "attn_ms_median": attn_ms_median}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -528,6 +590,7 @@ def run_ours(args):
             "pct_of_bf16_peak": 100.0 * value / peak,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clk,
             "gpu_launches": 2 * args.steps, "permutation": perm, "swa_comparison": swa,
+            "other_configs": others,
         }
         print(json.dumps(line))
     if world > 1:

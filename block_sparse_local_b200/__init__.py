@@ -11,6 +11,7 @@ Method (STA README "Sliding Tile Atteniton Kernel", section Usage):
 tokens), tiles of (6, 8, 8) tokens, ``window_size`` in tiles.
 """
 import ctypes
+import functools
 import os
 
 import torch
@@ -97,6 +98,21 @@ def lib():
     return L
 
 
+def _ranged(fn):
+    """NVTX range "sta.<name>" around a public call, so that a profiler's
+    timeline shows which library call launched which kernels."""
+    name = "sta." + fn.__name__
+
+    @functools.wraps(fn)
+    def wrapper(*args, **kwargs):
+        torch.cuda.nvtx.range_push(name)
+        try:
+            return fn(*args, **kwargs)
+        finally:
+            torch.cuda.nvtx.range_pop()
+    return wrapper
+
+
 def _check(code, where):
     if code != 0:
         raise StaError(code, where)
@@ -126,6 +142,7 @@ def _check_qkv(*ts):
             raise ValueError("tensors must be contiguous bf16 CUDA tensors")
 
 
+@_ranged
 def tile_reorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
     """[B, heads, S, d] raster order -> tile order (text rows unchanged)."""
     _check_qkv(x)
@@ -137,6 +154,7 @@ def tile_reorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
     return out
 
 
+@_ranged
 def tile_unreorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
     """Inverse of tile_reorder."""
     _check_qkv(x)
@@ -148,6 +166,7 @@ def tile_unreorder(x, video_shape, tile=(6, 8, 8), has_text=True, out=None):
     return out
 
 
+@_ranged
 def build_kv_tile_lists(window_size, video_shape, tile=(6, 8, 8), text_length=0,
                         has_text=True, max_k=None, device="cuda"):
     """Per-head KV tile lists: (counts [heads, NQ], ids [heads, NQ, max_k])."""
@@ -166,6 +185,7 @@ def build_kv_tile_lists(window_size, video_shape, tile=(6, 8, 8), text_length=0,
     return counts, ids
 
 
+@_ranged
 def forward(q, k, v, window_size, text_length, has_text, video_shape,
             tile=(6, 8, 8), out=None, return_lse=False):
     """STA attention on TILE-ordered q, k, v [B, heads, S, d] (bf16)."""
@@ -186,6 +206,7 @@ def forward(q, k, v, window_size, text_length, has_text, video_shape,
     return out
 
 
+@_ranged
 def forward_noalloc(q, k, v, window_size, text_length, has_text, video_shape,
                     tile=(6, 8, 8), out=None):
     """Like forward(), through sta_forward_noalloc: the library allocates no
@@ -202,6 +223,7 @@ def forward_noalloc(q, k, v, window_size, text_length, has_text, video_shape,
     return out
 
 
+@_ranged
 def forward_raster(q, k, v, window_size, text_length, has_text, video_shape,
                    tile=(6, 8, 8), out=None, return_lse=False):
     """STA attention on RASTER-ordered q, k, v with the permutation fused into
@@ -219,6 +241,7 @@ def forward_raster(q, k, v, window_size, text_length, has_text, video_shape,
     return (out, lse) if return_lse else out
 
 
+@_ranged
 def backward(q, k, v, out, dout, lse, window_size, text_length, has_text, video_shape,
              tile=(6, 8, 8)):
     """Gradients (dq, dk, dv) of forward() on TILE-ordered tensors; lse from
@@ -268,6 +291,7 @@ class TileReorderFunction(torch.autograd.Function):
         return f(g.contiguous(), video_shape, tile, has_text), None, None, None, None
 
 
+@_ranged
 def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
                            video_shape=(30, 48, 80), tile=(6, 8, 8), fused=True):
     """README-style call on RASTER-ordered q, k, v.
@@ -299,6 +323,7 @@ def sliding_tile_attention(q, k, v, window_size, text_length, has_text=True,
     return tile_unreorder(ot, video_shape, tile, has_text)
 
 
+@_ranged
 def sliding_tile_attention_host(q, k, v, window_size, text_length, has_text=True,
                                 video_shape=(30, 48, 80), tile=(6, 8, 8), out=None,
                                 device=None, blocking=True, chunk_bytes=0):
@@ -340,6 +365,7 @@ def sliding_tile_attention_host(q, k, v, window_size, text_length, has_text=True
     return out
 
 
+@_ranged
 def swa3d_forward(q, k, v, window_tokens, text_length, has_text, video_shape,
                   tile=(6, 8, 8), out=None):
     """Token-level 3-D sliding-window attention on RASTER-ordered q, k, v:
@@ -358,6 +384,7 @@ def swa3d_forward(q, k, v, window_tokens, text_length, has_text, video_shape,
 ORDERS = {"raster": 0, "hilbert": 1}
 
 
+@_ranged
 def hilbert_reorder(x, n, to_hilbert=True, out=None):
     """[B, heads, n*n, d] rows between raster and Hilbert order (bit-exact)."""
     _check_qkv(x)
@@ -368,6 +395,7 @@ def hilbert_reorder(x, n, to_hilbert=True, out=None):
     return out
 
 
+@_ranged
 def build_slide_block_lists(n, window, order="hilbert", device="cuda"):
     """(counts [nb], ids [nb, nb], classes [nb, nb]) of 2-D slide attention."""
     nb = n * n // 128
@@ -380,6 +408,7 @@ def build_slide_block_lists(n, window, order="hilbert", device="cuda"):
     return counts, ids, cls
 
 
+@_ranged
 def slide2d_forward(q, k, v, n, window, order="hilbert", out=None):
     """Block-sparse 2-D slide attention on q, k, v stored in `order`."""
     _check_qkv(q, k, v)
@@ -391,6 +420,7 @@ def slide2d_forward(q, k, v, n, window, order="hilbert", out=None):
     return out
 
 
+@_ranged
 def slide_attention_2d(q, k, v, n, window, order="hilbert"):
     """Raster-ordered in and out; with order='hilbert' the tokens are reordered
     along the Hilbert curve, attended block-sparsely, and put back."""
@@ -401,6 +431,7 @@ def slide_attention_2d(q, k, v, n, window, order="hilbert"):
     return hilbert_reorder(oh, n, False)
 
 
+@_ranged
 def swa_forward(q, k, v, window, causal=True, out=None):
     """Token-level causal sliding-window attention, GQA: q [B,hq,S,d], k,v [B,hkv,S,d]."""
     _check_qkv(q, k, v)
