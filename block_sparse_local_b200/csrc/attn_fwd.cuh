@@ -24,9 +24,12 @@
 //               O_i += P_i V (TS: P from TMEM, V from shared memory, N=d),
 //               ping-ponging the two slots so the tensor pipe works on one
 //               slot while the other slot's softmax runs.
-//   warps 2..   softmax, 4 * kSplit warps per slot: kSplit warps share each
-//               query row (TMEM lane), each with 128 / kSplit of its scores;
-//               exponentials two at a time with packed f32x2 arithmetic (a
+//   warps 2..   softmax, 8 warps per slot, two per TMEM lane quarter, each
+//               warp on 16 of the quarter's 32 query rows (TMEM lanes) with
+//               two threads per row (lanes t and t + 16), each thread with 64
+//               of the row's 128 scores, so the row's max and sum are one
+//               warp shuffle away; exponentials two at a time with packed
+//               f32x2 arithmetic (a
 //               share of them on the FMA pipe) against the running max, the
 //               block max taken in the same loop; they update the running
 //               max / sum, write bf16 P over the first half of their own
@@ -46,12 +49,10 @@ namespace sta {
 
 constexpr int kBM = 128;        // query rows per block (MMA M)
 constexpr int kBN = 128;        // keys per block
-// Warps that share one query row's softmax (each takes 128 / kSplit score
-// columns of the row); the two slots' softmax use 8 * kSplit warps.
-#ifndef STA_SOFTMAX_SPLIT
-#define STA_SOFTMAX_SPLIT 2
-#endif
-constexpr int kSplit = STA_SOFTMAX_SPLIT;
+// Threads that share one query row's softmax (each takes 128 / kSplit score
+// columns of the row, two lanes of one warp); the two slots' softmax use
+// 8 * kSplit warps.
+constexpr int kSplit = 2;
 
 constexpr int kFwdThreads = 64 + 256 * kSplit;
 constexpr int kWarpTma = 0;
@@ -115,9 +116,7 @@ struct FwdCfg {
   static constexpr int kKOff = kQOff + 2 * kBlockBytes;
   static constexpr int kVOff = kKOff + kKStages * kBlockBytes;
   static constexpr int kBarOff = kVOff + kVStages * kBlockBytes;
-  static constexpr int kRedOff = kBarOff + 512;   // row-max / row-sum exchange
-  static constexpr int kRedBytes = 2 * 2 * 2 * kBM * 4;
-  static constexpr int kSmemBytes = kRedOff + kRedBytes + 1024;  // + 1024-byte align
+  static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + 1024-byte align
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kOCol = 256;
 };
@@ -329,8 +328,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* p_full = s_full + 2;      // [2]
   uint64_t* o_full = p_full + 2;      // [2]
   uint64_t* mma_done = o_full + 2;
-  uint64_t* xbar = mma_done + 1;      // [2 slots][4 lane quarters] exchange
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(xbar + 8);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -350,7 +348,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&o_full[i], 1);
     }
     mbar_init(mma_done, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&xbar[i], kSplit);   // one arrival per warp
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
     fence_mbar_init();
   }
@@ -497,29 +494,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    // kSplit warps share each query row: warp k of the softmax warps serves
-    // slot k / (4 kSplit), column half (k / 4) % kSplit, TMEM lane quarter
-    // warp % 4.  With kSplit = 2 the halves exchange their partial row max
-    // every block (and their partial sums once, at the end) through shared
-    // memory behind an mbarrier.
+    // Warp k of the softmax warps serves slot k / 8, TMEM lane quarter
+    // warp % 4 and, in it, the 16 rows of row half (k / 4) % 2; lanes t and
+    // t + 16 share row t % 16, lane t + 16 taking columns 64-127 (the
+    // .16x32bx2 TMEM accesses), so the two halves of a row meet through a
+    // warp shuffle.
     constexpr int kCols = kBN / kSplit;       // score columns per thread
     constexpr int kOCols = D / kSplit;        // output columns per thread
     const int ks = warp - kWarpSoftmax0;
-    const int slot = ks / (4 * kSplit);
-    const int half = (ks / 4) % kSplit;
+    const int slot = ks / 8;
+    const int rh = (ks / 4) % 2;              // row half of the lane quarter
+    const int half = lane >> 4;               // column half of the row
     const int sub = warp & 3;                 // TMEM lane quarter of this warp
-    const int r = sub * 32 + lane;            // query row inside the block
-    float* red = reinterpret_cast<float*>(smem + C::kRedOff);   // [2][2][2][128]
-    uint64_t* xb = &xbar[slot * 4 + sub];
-    (void)red;
-    (void)xb;
+    const int r = sub * 32 + rh * 16 + (lane & 15);   // query row inside the block
     if (!skip && (slot == 0 || two)) {
-      const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u) + half * kCols;
+      const uint32_t lane_off = static_cast<uint32_t>(sub * 32 + rh * 16) << 16;
+      // this warp's 16 lanes; the column half follows from the split offset
+      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u);
       // P over the first half of this thread's own score columns, so no
-      // warp overwrites scores that another warp has still to read
-      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u) + half * kCols;
-      const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0) + half * kOCols;
+      // thread overwrites scores that another has still to read
+      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u);
+      const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0);
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY;   // running max, log2 units of the scaled scores
       float l_run = 0.f;         // this thread's part of the row sum
@@ -568,7 +563,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         auto load_scores = [&]() {
           uint32_t sr[kCols];
 #pragma unroll
-          for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_LD32(t_s + cc * 32, (sr + cc * 32));
+          for (int cc = 0; cc < kCols / 32; ++cc) tmem_ld_half32<kCols>(t_s + cc * 32, sr + cc * 32);
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < kCols; ++c) s[c] = __uint_as_float(sr[c]);
@@ -657,16 +652,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           return fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
         };
-        // the halves of a row agree on the block's max through shared memory
-        float* rb = red + ((j & 1) * 2 + slot) * 2 * kBM;
+        // the halves of a row (lanes t, t + 16) agree on the block's max
         auto exchange_max = [&](float& mx) {
-          if constexpr (kSplit == 2) {
-            rb[half * kBM + r] = mx;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(xb);
-            if (!mbar_wait_warp(xb, j & 1, abort_flag)) return false;
-            mx = fmaxf(mx, rb[(half ^ 1) * kBM + r]);
-          }
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
           return true;
         };
         // Reference of the exponent: the running max (log2 units), raised
@@ -711,17 +699,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         // bf16 P over the first half of this thread's own score columns
 #pragma unroll
-        for (int cc = 0; cc < kCols / 32; ++cc) STA_TMEM_ST16(t_p + cc * 16, (pk + cc * 16));
+        for (int cc = 0; cc < kCols / 32; ++cc) tmem_st_half16<kCols>(t_p + cc * 16, pk + cc * 16);
         l_run += lsum;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
 #pragma unroll
           for (int cc = 0; cc < kOCols / 32; ++cc) {
             uint32_t o[32];
-            STA_TMEM_LD32(t_o + cc * 32, o);
+            tmem_ld_half32<kOCols>(t_o + cc * 32, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            STA_TMEM_ST32(t_o + cc * 32, o);
+            tmem_st_half32<kOCols>(t_o + cc * 32, o);
           }
         }
         tmem_wait_st();
@@ -731,16 +719,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (done && mbar_wait_warp(&o_full[slot], 0, abort_flag)) {
         tc_fence_after();
-        bool ok = true;
-        if constexpr (kSplit == 2) {
-          float* rb = red + ((n & 1) * 2 + slot) * 2 * kBM;
-          rb[half * kBM + r] = l_run;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(xb);
-          ok = mbar_wait_warp(xb, n & 1, abort_flag);
-          if (ok) l_run += rb[(half ^ 1) * kBM + r];
-        }
-        if (ok) {
+        l_run += __shfl_xor_sync(0xffffffffu, l_run, 16);
+        {
           const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
           int qrow = (slot ? item.q1 : item.q0) + r;
           if constexpr (R) qrow = raster_row(p, qrow);
@@ -749,7 +729,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
           for (int cc = 0; cc < kOCols / 32; ++cc) {
             uint32_t o[32];
-            STA_TMEM_LD32(t_o + cc * 32, o);
+            tmem_ld_half32<kOCols>(t_o + cc * 32, o);
             tmem_wait_ld();
             uint32_t pk[16];
 #pragma unroll
