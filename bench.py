@@ -66,6 +66,10 @@ def parse():
                     help="run the workload with fewer heads (profiling captures only)")
     ap.add_argument("--backward-only", action="store_true",
                     help="time only the backward pass of the workload (profiling captures)")
+    ap.add_argument("--profile-workload", default=None,
+                    help="run only the forward of this named STA workload (raster order), "
+                         "--steps times after --warmup, for profiling captures; "
+                         "--heads keeps that many heads")
     return ap.parse_args()
 
 
@@ -310,6 +314,36 @@ def run_reference(args):
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line))
+    return 0
+
+
+def run_profile_workload(args):
+    """Forward of one named workload only (profiling captures of the d = 64
+    kernel and of the other shapes); prints its time, not a bench line."""
+    import dataclasses
+    import torch
+    import block_sparse_local_b200 as sta
+    from block_sparse_local_b200 import workloads
+    w = workloads.STA_WORKLOADS[args.profile_workload]
+    if args.heads is not None:
+        w = dataclasses.replace(w, heads=args.heads, windows=w.windows[:args.heads])
+    dev = torch.device("cuda", 0)
+    shape = (w.T, w.H, w.W)
+    q, k, v = workloads.sta_inputs(w, device=dev)
+    out = torch.empty_like(q)
+    for i in range(args.warmup + args.steps):
+        if i == args.warmup:
+            torch.cuda.synchronize(dev)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+        sta.forward_raster(q, k, v, w.windows, w.text_len, w.has_text, shape, w.tile, out=out)
+    b.record()
+    torch.cuda.synchronize(dev)
+    sta.device_status(dev)
+    ms = a.elapsed_time(b) / max(1, args.steps)
+    pairs = sta.retained_pairs(w.B, w.windows, shape, w.tile, w.text_len, w.has_text)
+    print(json.dumps({"profile_workload": w.name, "heads": w.heads, "ms": ms,
+                      "effective_tflops": 4.0 * w.d * pairs / (ms * 1e-3) / 1e12}))
     return 0
 
 
@@ -603,6 +637,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_workload is not None:
+        return run_profile_workload(args)
     return run_ours(args)
 
 
