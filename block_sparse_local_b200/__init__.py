@@ -16,7 +16,7 @@ import os
 
 import torch
 
-from .build import LIB_PATH
+from .build import DEBUG_LIB_PATH, LIB_PATH
 
 __all__ = [
     "StaError", "lib", "tile_reorder", "tile_unreorder", "build_kv_tile_lists",
@@ -28,7 +28,8 @@ __all__ = [
 ]
 
 STATUS = {0: "STA_OK", 1: "STA_ERR_INVALID_ARG", 2: "STA_ERR_UNSUPPORTED",
-          3: "STA_ERR_CUDA", 4: "STA_ERR_DEVICE_TIMEOUT", 5: "STA_ERR_SCRATCH_LIMIT"}
+          3: "STA_ERR_CUDA", 4: "STA_ERR_DEVICE_TIMEOUT", 5: "STA_ERR_SCRATCH_LIMIT",
+          6: "STA_ERR_DEVICE_BOUNDS"}
 
 EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_forward", "sta_forward_lse", "sta_swa_forward",
@@ -36,7 +37,7 @@ EXPORTED = ("sta_tile_reorder", "sta_tile_unreorder", "sta_build_kv_tile_lists",
             "sta_retained_pairs", "sta_forward_noalloc", "sta_forward_raster",
             "sta_swa3d_forward", "sta_debug_inject", "sta_hilbert_reorder",
             "sta_build_slide_block_lists", "sta_slide2d_forward", "sta_backward",
-            "sta_forward_raster_host", "sta_debug_pair_kernel")
+            "sta_forward_raster_host", "sta_debug_pair_kernel", "sta_debug_checks")
 
 
 class StaError(RuntimeError):
@@ -46,6 +47,7 @@ class StaError(RuntimeError):
 
 
 _LIB = None
+_DEBUG_LIB = None
 _P = ctypes.c_void_p
 _I = ctypes.c_int
 _I3 = ctypes.c_int * 3
@@ -54,13 +56,27 @@ _I3 = ctypes.c_int * 3
 def lib():
     """Loads libsta.so (built in-tree); raises if it is missing."""
     global _LIB
-    if _LIB is not None:
-        return _LIB
-    if not os.path.exists(LIB_PATH):
+    if _LIB is None:
+        _LIB = _load(LIB_PATH)
+    return _LIB
+
+
+def debug_lib():
+    """Loads libsta_debug.so, the build with device bounds checks (same entry
+    points; a failed check is reported by sta_device_status as
+    STA_ERR_DEVICE_BOUNDS); raises if it is missing."""
+    global _DEBUG_LIB
+    if _DEBUG_LIB is None:
+        _DEBUG_LIB = _load(DEBUG_LIB_PATH)
+    return _DEBUG_LIB
+
+
+def _load(path):
+    if not os.path.exists(path):
         raise RuntimeError(
-            f"{LIB_PATH} is missing: build it with "
+            f"{path} is missing: build it with "
             "`python -m block_sparse_local_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     geo = [_I, _I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int)]
     L.sta_tile_reorder.argtypes = [_P, _P] + geo + [_I, _P]
     L.sta_tile_unreorder.argtypes = [_P, _P] + geo + [_I, _P]
@@ -90,11 +106,11 @@ def lib():
     L.sta_retained_pairs.argtypes = [_I, _I, _I, _I, _I, ctypes.POINTER(ctypes.c_int),
                                      ctypes.POINTER(ctypes.c_int), _I, _I]
     L.sta_retained_pairs.restype = ctypes.c_int64
+    L.sta_debug_checks.argtypes = []
     for name in EXPORTED:
         fn = getattr(L, name)
         if name not in ("sta_status_string", "sta_shutdown", "sta_retained_pairs"):
             fn.restype = ctypes.c_int
-    _LIB = L
     return L
 
 

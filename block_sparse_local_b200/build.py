@@ -1,4 +1,5 @@
-"""Builds libsta.so in-tree for sm_100a with nvcc.
+"""Builds libsta.so (release) and libsta_debug.so (device bounds checks,
+STA_DEBUG=1) in-tree for sm_100a with nvcc.
 
     python -m block_sparse_local_b200.build [--verbose]
 
@@ -12,6 +13,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB_PATH = os.path.join(HERE, "libsta.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libsta_debug.so")
 SOURCES = [os.path.join(HERE, "csrc", "sta_lib.cu")]
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
                      ("device_ptx.cuh", "reorder.cuh", "tile_lists.cuh",
@@ -31,22 +33,32 @@ def command(out=LIB_PATH, extra=()):
             "-I" + os.path.join(ROOT, "include"), *extra, "-o", out, *SOURCES]
 
 
-def up_to_date():
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path=LIB_PATH):
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(f) <= t for f in DEPENDS)
 
 
-def build(force=False, verbose=False):
-    if not force and up_to_date():
-        return LIB_PATH
-    cmd = command(extra=("-Xptxas", "-v") if verbose else ())
-    res = subprocess.run(cmd, capture_output=True, text=True)
-    if verbose or res.returncode != 0:
-        sys.stderr.write(res.stdout + res.stderr)
-    if res.returncode != 0:
-        raise RuntimeError("nvcc failed building libsta.so")
+def build(force=False, verbose=False, debug=True):
+    """Builds libsta.so and (debug=True) libsta_debug.so, in parallel."""
+    jobs = [(LIB_PATH, ())]
+    if debug:
+        jobs.append((DEBUG_LIB_PATH, ("-DSTA_DEBUG=1",)))
+    procs = []
+    for path, defs in jobs:
+        if not force and up_to_date(path):
+            continue
+        extra = tuple(defs) + (("-Xptxas", "-v") if verbose else ())
+        procs.append((path, subprocess.Popen(command(out=path, extra=extra),
+                                             stdout=subprocess.PIPE, stderr=subprocess.PIPE,
+                                             text=True)))
+    for path, proc in procs:
+        out, err = proc.communicate()
+        if verbose or proc.returncode != 0:
+            sys.stderr.write(out + err)
+        if proc.returncode != 0:
+            raise RuntimeError(f"nvcc failed building {os.path.basename(path)}")
     return LIB_PATH
 
 

@@ -53,6 +53,8 @@ struct BwdParams {
   const float* neg_delta; // [rows] minus D
   __nv_bfloat16* out_a;   // dQ (dQ kernel) or dK (dK/dV kernel)
   __nv_bfloat16* out_b;   // dV (dK/dV kernel)
+  int dbg_rows;           // rows of every [rows, d] tensor (debug-build bounds checks)
+  int dbg_lists;          // rows of the lists
 };
 
 template <int D>
@@ -195,11 +197,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const WorkItem item = p.items[blockIdx.x];
+  // debug build: the item and its list lie inside the arrays they index
+  const bool item_ok = dbg_ok(item.q0 >= 0 && item.q0 + 128 <= p.dbg_rows &&
+                              item.kv_base >= 0 && item.kv_base < p.dbg_rows &&
+                              item.list >= 0 && item.list < p.dbg_lists) &&
+                       dbg_ok(p.counts[item.list] >= 0 && p.counts[item.list] <= p.max_k);
   // stream: key blocks of the query block (dQ) or query blocks of the key block (dK/dV)
-  const int cnt = p.counts[item.list];
-  const int* ids = p.ids + static_cast<size_t>(item.list) * p.max_k;
+  const int cnt = item_ok ? p.counts[item.list] : 0;
+  const int* ids = p.ids + static_cast<size_t>(item_ok ? item.list : 0) * p.max_k;
   const int nvid = (cnt - p.text_sentinel) * p.tile_blocks;
-  const int n = nvid + (p.text_sentinel ? p.text_blocks : 0);
+  const int n = item_ok ? nvid + (p.text_sentinel ? p.text_blocks : 0) : 0;
   auto stream_row = [&](int j) {
     if (j < nvid) {
       const int t = j / p.tile_blocks;
@@ -263,6 +270,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int st = j % ST;
         if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
         const int row = stream_row(j);
+        if (!dbg_ok(row >= 0 && row + 128 <= p.dbg_rows)) {
+          *abort_flag = 1;
+          break;
+        }
         uint8_t* base = smem + C::kStream + st * C::kStageBytes;
         if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + 1024);
         if (!is_vec) {

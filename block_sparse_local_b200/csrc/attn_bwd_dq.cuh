@@ -101,11 +101,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const WorkItem item = p.items[blockIdx.x];
+  // debug build: the item and its list lie inside the arrays they index
+  const bool item_ok = dbg_ok(item.q0 >= 0 && item.q0 + 128 <= p.dbg_rows &&
+                              item.kv_base >= 0 && item.kv_base < p.dbg_rows &&
+                              item.list >= 0 && item.list < p.dbg_lists) &&
+                       dbg_ok(p.counts[item.list] >= 0 && p.counts[item.list] <= p.max_k);
   // the query block's key blocks: video tiles of its list, then the text block
-  const int cnt = p.counts[item.list];
-  const int* ids = p.ids + static_cast<size_t>(item.list) * p.max_k;
+  const int cnt = item_ok ? p.counts[item.list] : 0;
+  const int* ids = p.ids + static_cast<size_t>(item_ok ? item.list : 0) * p.max_k;
   const int nvid = (cnt - p.text_sentinel) * p.tile_blocks;
-  const int n = nvid + (p.text_sentinel ? p.text_blocks : 0);
+  const int n = item_ok ? nvid + (p.text_sentinel ? p.text_blocks : 0) : 0;
   auto key_row = [&](int j) {
     if (j < nvid) {
       const int t = j / p.tile_blocks;
@@ -161,9 +166,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       for (int j = 0; j < n; ++j) {
         const int st = j % nst;
         if (j >= nst && !mbar_wait(&empty[st], ((j / nst) - 1) & 1, abort_flag)) break;
+        const int row = key_row(j);
+        if (!dbg_ok(row >= 0 && row + 128 <= p.dbg_rows)) {
+          *abort_flag = 1;
+          break;
+        }
         if (pn == 0) mbar_arrive_expect_tx(&full[st], C::kBlockBytes);
         tma_load_2d_hint(base + st * C::kBlockBytes + pn * C::kPanelBytes, map, &full[st],
-                         pn * 64, key_row(j), pol);
+                         pn * 64, row, pol);
       }
       __syncwarp((1u << (2 * kPanels)) - 1u);
       // Leave no copy in flight: wait for the last load of every stage.

@@ -103,7 +103,28 @@ struct FwdParams {
   __nv_bfloat16* out;
   float* lse;
   RasterGeom rg;      // used when the kernel runs on raster-ordered tensors
+  // extents for the bounds checks of the debug build
+  int dbg_rows_q;     // rows of q and out in the [rows, d] view
+  int dbg_rows_kv;    // rows of k and v
+  int dbg_lists;      // rows of the key-block lists (kSta, kSwa3d, kSlide2d)
 };
+
+// Debug build: the work item and its key-block list are inside the arrays
+// they index (checked once per CTA before anything is loaded).
+template <Mode M>
+__device__ __forceinline__ bool item_in_bounds(const FwdParams& p, const WorkItem& it) {
+  bool ok = it.q0 >= 0 && it.q0 + kBM <= p.dbg_rows_q;
+  ok = ok && (it.q1 < 0 || it.q1 + kBM <= p.dbg_rows_q);
+  ok = ok && it.kv_base >= 0 && it.kv_base < p.dbg_rows_kv;
+  if constexpr (M != Mode::kSwa) {
+    ok = ok && it.list >= 0 && it.list < p.dbg_lists;
+    if (ok) {
+      const int cnt = p.counts[it.list];
+      ok = cnt >= 0 && cnt <= p.max_k;
+    }
+  }
+  return ok;
+}
 
 template <int D>
 struct FwdCfg {
@@ -348,7 +369,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&o_full[i], 1);
     }
     mbar_init(mma_done, 1);
-    *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
+    bool bad = false;
+    if constexpr (STA_DEBUG) bad = !dbg_ok(item_in_bounds<M>(p, item));
+    *abort_flag = (error_raised() || n <= 0 || bad) ? 1 : 0;
     fence_mbar_init();
   }
   if (warp == kWarpTma && lane == 0) {
@@ -403,6 +426,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int st = j % NST;
         if (j >= NST && !mbar_wait(&empty[st], ((j / NST) - 1) & 1, abort_flag)) break;
         const int row = seq_row<M>(p, seq, j);
+        if (!dbg_ok(row >= 0 && row + kBN <= p.dbg_rows_kv)) {
+          *abort_flag = 1;                 // the other roles give up at their next poll
+          break;
+        }
         if (pn == 0) mbar_arrive_expect_tx(&full[st], C::kBlockBytes);
         load_panel<D, R>(base + st * C::kBlockBytes, m2, m5, &full[st], row, p, pol_kv, pn);
       }
@@ -724,6 +751,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
           int qrow = (slot ? item.q1 : item.q0) + r;
           if constexpr (R) qrow = raster_row(p, qrow);
+          const bool row_ok = dbg_ok(qrow >= 0 && qrow < p.dbg_rows_q);
+          if (!row_ok) qrow = 0;             // debug build: the stores below are skipped
           uint4* dst = reinterpret_cast<uint4*>(p.out + static_cast<size_t>(qrow) * D +
                                                 half * kOCols);
 #pragma unroll
@@ -736,12 +765,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int e = 0; e < 16; ++e)
               pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * inv,
                                   __uint_as_float(o[2 * e + 1]) * inv);
+            if (row_ok) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
-                                            pk[4 * v4 + 3]);
+              for (int v4 = 0; v4 < 4; ++v4)
+                dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
+                                              pk[4 * v4 + 3]);
+            }
           }
-          if (p.lse != nullptr && half == 0) {
+          if (p.lse != nullptr && half == 0 && row_ok) {
             const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
             p.lse[qrow] = (m_use + __log2f(l_run)) * 0.69314718055994531f;
           }

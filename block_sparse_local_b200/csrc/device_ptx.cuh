@@ -41,6 +41,30 @@ __device__ __forceinline__ void raise_error(unsigned int bit) {
   atomicOr(&g_error_word, bit);
 }
 
+// Debug build (libsta_debug.so, compiled with -DSTA_DEBUG=1): bounds checks
+// of the index arithmetic that feeds global loads and stores, TMA coordinates
+// and work-plan reads.  A failed check records bit 1 of the device error word
+// (sta_device_status() then reports STA_ERR_DEVICE_BOUNDS) and the caller
+// skips the access; nothing traps.  In the release build every check is
+// true at compile time and costs nothing.
+#ifndef STA_DEBUG
+#define STA_DEBUG 0
+#endif
+constexpr unsigned int kErrTimeout = 1u;
+constexpr unsigned int kErrBounds = 2u;
+
+__device__ __forceinline__ bool dbg_ok(bool in_bounds) {
+#if STA_DEBUG
+  if (!in_bounds) {
+    raise_error(kErrBounds);
+    return false;
+  }
+#else
+  (void)in_bounds;
+#endif
+  return true;
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),

@@ -15,6 +15,8 @@
 // contiguous rows (runs of cw rows are contiguous on the raster side).
 #pragma once
 
+#include "device_ptx.cuh"
+
 #include <cstdint>
 
 namespace sta {
@@ -65,7 +67,9 @@ __global__ void __launch_bounds__(256) tile_permute_kernel(
     const int rows = g.S - g.Lv;
     const int n = rows * kVec;
     const size_t base = (slice_base + g.Lv) * kVec;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) out[base + i] = in[base + i];
+    const size_t total = static_cast<size_t>(gridDim.y) * g.S * kVec;
+    for (int i = threadIdx.x; i < n; i += blockDim.x)
+      if (dbg_ok(base + i < total)) out[base + i] = in[base + i];
     return;
   }
   const int tw = tile % g.NW;
@@ -93,13 +97,16 @@ __global__ void __launch_bounds__(256) tile_permute_kernel(
         const size_t tiled = tile_row0 + row;
         const size_t src = (to_tile ? raster : tiled) * kVec + vec;
         dst[u] = (to_tile ? tiled : raster) * kVec + vec;
-        v[u] = __ldg(in + src);
+        const size_t total = static_cast<size_t>(gridDim.y) * g.S * kVec;
+        v[u] = dbg_ok(src < total) ? __ldg(in + src) : make_uint4(0u, 0u, 0u, 0u);
+        if (!dbg_ok(dst[u] < total)) dst[u] = total;   // marks the store as skipped
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int i = base + u * blockDim.x;
-      if (i < n) out[dst[u]] = v[u];
+      if (i < n && (!STA_DEBUG || dst[u] < static_cast<size_t>(gridDim.y) * g.S * kVec))
+        out[dst[u]] = v[u];
     }
   }
 }

@@ -635,6 +635,9 @@ sta_status forward_impl(const void* q, const void* k, const void* v, void* out, 
   FwdParams prm{};
   prm.items = d_items;
   prm.item_off = pair ? d_off : nullptr;
+  prm.dbg_rows_q = static_cast<int>(total_rows);
+  prm.dbg_rows_kv = static_cast<int>(total_rows);
+  prm.dbg_lists = cls.nclass * NQ;
   prm.counts = d_counts;
   prm.ids = d_ids;
   prm.max_k = max_k;
@@ -993,6 +996,9 @@ sta_status forward_noalloc_impl(const void* q, const void* k, const void* v, voi
   FwdParams prm{};
   prm.items = d_items;
   prm.item_off = nullptr;
+  prm.dbg_rows_q = static_cast<int>(total_rows);
+  prm.dbg_rows_kv = static_cast<int>(total_rows);
+  prm.dbg_lists = cls.nclass * NQ;
   prm.counts = d_counts;
   prm.ids = d_ids;
   prm.max_k = max_k;
@@ -1259,6 +1265,8 @@ sta_status backward_impl(const void* q, const void* k, const void* v, const void
   prm.scale = static_cast<float>(1.0 / std::sqrt(double(d)));
   prm.neg_lse2 = neg_lse2;
   prm.neg_delta = neg_delta;
+  prm.dbg_rows = static_cast<int>(rows);
+  prm.dbg_lists = cls.nclass * NQ;
   // dQ: forward lists, text key blocks with valid keys
   prm.items = qitems;
   prm.counts = fc;
@@ -1298,6 +1306,8 @@ const char* sta_status_string(sta_status s) {
     case STA_ERR_DEVICE_TIMEOUT: return "STA_ERR_DEVICE_TIMEOUT: a device wait gave up";
     case STA_ERR_SCRATCH_LIMIT:
       return "STA_ERR_SCRATCH_LIMIT: problem needs more than the fixed no-alloc scratch";
+    case STA_ERR_DEVICE_BOUNDS:
+      return "STA_ERR_DEVICE_BOUNDS: a device bounds check failed (debug build)";
   }
   return "STA_ERR_UNKNOWN";
 }
@@ -1427,6 +1437,8 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   FwdParams prm{};
   std::memset(&prm, 0, sizeof(prm));
   prm.items = d_items;
+  prm.dbg_rows_q = static_cast<int>(qrows);
+  prm.dbg_rows_kv = static_cast<int>(int64_t(B) * hkv * S);
   prm.window = window;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(double(d)));
   prm.out = static_cast<__nv_bfloat16*>(out);
@@ -1437,6 +1449,8 @@ sta_status sta_swa_forward(const void* q, const void* k, const void* v, void* ou
   if (s != STA_OK) return s;
   return order_end(ws.order, st);
 }
+
+int sta_debug_checks(void) { return STA_DEBUG ? 1 : 0; }
 
 sta_status sta_debug_pair_kernel(int pair) {
   if (pair != 0 && pair != 1) return STA_ERR_INVALID_ARG;
@@ -1570,6 +1584,9 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v, void
   FwdParams prm{};
   std::memset(&prm, 0, sizeof(prm));
   prm.items = items;
+  prm.dbg_rows_q = static_cast<int>(rows);
+  prm.dbg_rows_kv = static_cast<int>(rows);
+  prm.dbg_lists = np;
   prm.counts = counts;
   prm.ids = ids;
   prm.max_k = nb;
@@ -1612,7 +1629,8 @@ sta_status sta_device_status(void* stream) {
   if (word != 0) {
     const unsigned int zero = 0;
     STA_CUDA_TRY(cudaMemcpyToSymbol(sta::g_error_word, &zero, sizeof(zero)));
-    return STA_ERR_DEVICE_TIMEOUT;
+    // a failed bounds check (debug build) is the cause of any later time-outs
+    return (word & sta::kErrBounds) ? STA_ERR_DEVICE_BOUNDS : STA_ERR_DEVICE_TIMEOUT;
   }
   if (cudaGetLastError() != cudaSuccess) return STA_ERR_CUDA;
   return STA_OK;

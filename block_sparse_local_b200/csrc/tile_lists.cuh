@@ -13,6 +13,8 @@
 // the sentinel.  Unused slots up to max_k are -1.
 #pragma once
 
+#include "device_ptx.cuh"
+
 namespace sta {
 
 constexpr int kMaxWindowClasses = 256;
@@ -82,11 +84,13 @@ __global__ void __launch_bounds__(128) kv_tile_list_kernel(
     }
     for (int t = st; t < st + et; ++t)
       for (int h = sh; h < sh + eh; ++h)
-        for (int w = sw; w < sw + ew; ++w) out[n++] = (t * g.NH + h) * g.NW + w;
+        for (int w = sw; w < sw + ew; ++w)
+          if (dbg_ok(n < g.max_k)) out[n++] = (t * g.NH + h) * g.NW + w;
   } else {
-    for (int t = 0; t < g.NV; ++t) out[n++] = t;
+    for (int t = 0; t < g.NV; ++t)
+      if (dbg_ok(n < g.max_k)) out[n++] = t;
   }
-  if (g.text_block) out[n++] = g.NV;
+  if (g.text_block && dbg_ok(n < g.max_k)) out[n++] = g.NV;
   counts[gid] = n;
   for (int i = n; i < g.max_k; ++i) out[i] = -1;
 }

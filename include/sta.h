@@ -51,8 +51,9 @@ typedef enum sta_status {
                                  tile volume not a multiple of 128, not sm_100   */
   STA_ERR_CUDA = 3,           /* a CUDA runtime / driver call failed             */
   STA_ERR_DEVICE_TIMEOUT = 4, /* a bounded device wait gave up (see above)       */
-  STA_ERR_SCRATCH_LIMIT = 5   /* sta_forward_noalloc: the problem needs more than
+  STA_ERR_SCRATCH_LIMIT = 5,  /* sta_forward_noalloc: the problem needs more than
                                  STA_NOALLOC_SCRATCH_BYTES of scratch            */
+  STA_ERR_DEVICE_BOUNDS = 6   /* debug build only: a device bounds check failed  */
 } sta_status;
 
 /* Text block size (README Usage: the text block is padded to 256 tokens). */
@@ -270,10 +271,22 @@ sta_status sta_slide2d_forward(const void* q, const void* k, const void* v,
                                void* out, int B, int heads, int d, int n,
                                int window, int order, void* stream);
 
-/* Synchronises `stream`, returns STA_ERR_DEVICE_TIMEOUT if any kernel of this
- * library recorded a gave-up wait since the last call (and clears it), else
- * STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
+/* Synchronises `stream`, returns STA_ERR_DEVICE_BOUNDS if a kernel of the
+ * debug build recorded a failed bounds check, else STA_ERR_DEVICE_TIMEOUT if
+ * any kernel of this library recorded a gave-up wait since the last call (and
+ * clears the record), else STA_ERR_CUDA on a pending CUDA error, else STA_OK. */
 sta_status sta_device_status(void* stream);
+
+/*
+ * sta_debug_checks - 1 in the debug build of the library (libsta_debug.so,
+ * compiled with STA_DEBUG=1), 0 in the release build (libsta.so).  No
+ * passage of the pages corresponds to it.  The debug build checks, on the
+ * device, that every work item, key-block list entry, TMA row coordinate
+ * and output / gradient row lies inside the arrays it indexes; a failed
+ * check records STA_ERR_DEVICE_BOUNDS for sta_device_status() and skips the
+ * access (nothing traps).  Same entry points, arguments and results.
+ */
+int sta_debug_checks(void);
 
 /*
  * sta_debug_inject - fault injection for tests; no passage of the pages

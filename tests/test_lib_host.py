@@ -42,6 +42,17 @@ def test_library_exports_every_declared_symbol(L):
     assert set(_declared()) == set(sta.EXPORTED)
 
 
+def test_debug_build_loads_with_every_symbol_and_its_checks_compiled_in(L):
+    # libsta_debug.so is the same library with the device bounds checks
+    # (STA_DEBUG=1); sta_debug_checks() tells the two builds apart
+    LD = sta.debug_lib()
+    for name in _declared():
+        assert hasattr(LD, name), name
+    assert LD.sta_debug_checks() == 1
+    assert L.sta_debug_checks() == 0
+    assert LD.sta_status_string(6).decode().startswith("STA_ERR_DEVICE_BOUNDS")
+
+
 def test_status_strings(L):
     for code, name in sta.STATUS.items():
         assert L.sta_status_string(code).decode().startswith(name)
