@@ -67,6 +67,13 @@ struct PairCfg {
 constexpr int kWarpKLoad = 0;
 constexpr int kWarpVLoad = 18;
 constexpr int kLoadStreams = 4;   // load streams (lanes) per operand panel
+// A stream waits for the release of the stage it is about to fill by phase
+// parity, which is only unambiguous while the stream is at most one phase
+// ahead of that stage's barrier.  With more streams than stages a stream can
+// reach block g + streams while block g (same stage, another phase) has not
+// even landed, pass the parity wait early and load into a stage in use.
+static_assert(kLoadStreams <= PairCfg::KST && kLoadStreams <= PairCfg::VST,
+              "at most one load stream per ring stage");
 constexpr int kPairThreads = 19 * 32;
 
 // Q K^T into score buffer `b` (SS pair MMA, M = 256, N = 128 keys, K = d).
