@@ -139,7 +139,11 @@ struct FwdCfg {
   static constexpr int kBarOff = kVOff + kVStages * kBlockBytes;
   static constexpr int kSmemBytes = kBarOff + 512 + 1024;  // + 1024-byte align
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kOCol = 256;
+  // Score buffers of 128 columns: one per slot at d = 128 (S0, S1, then
+  // O0, O1 fill the 512 columns); at d = 64 the two 64-column O's leave room
+  // for a pool of three, so a slot's next Q K^T can run before its P V.
+  static constexpr int kSBuf = D == 64 ? 3 : 2;
+  static constexpr uint32_t kOCol = kSBuf * 128;
 };
 
 // Key-block sequence of one work item, identical for all roles.
@@ -290,10 +294,12 @@ __device__ __forceinline__ int raster_row(const FwdParams& p, int row) {
   return slice * g.S + ((tt * g.ct + it) * g.H + th * g.ch + ih) * g.W + tw * g.cw + iw;
 }
 
-// S_slot = Q_slot K^T over d (SS; K block in stage ks).  TMEM: S0 at column
-// 0, S1 at 128.  All operands warp-uniform, accumulate flags constant.
+// S_slot = Q_slot K^T over d (SS; K block in stage ks) into the score
+// buffer at TMEM column scol.  All operands warp-uniform, accumulate flags
+// constant.
 template <int D, int SLOT>
-__device__ __forceinline__ void fwd_issue_s(uint32_t tm, uint64_t dq, uint64_t dk, int ks) {
+__device__ __forceinline__ void fwd_issue_s(uint32_t tm, uint64_t dq, uint64_t dk, int ks,
+                                            uint32_t scol) {
   using C = FwdCfg<D>;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false);
   const uint64_t qa = dq + ((SLOT * C::kBlockBytes) >> 4);
@@ -301,17 +307,18 @@ __device__ __forceinline__ void fwd_issue_s(uint32_t tm, uint64_t dq, uint64_t d
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
-    umma_ss(tm + SLOT * 128u, qa + off, ka + off, kIdesc, kk > 0 ? 1u : 0u);
+    umma_ss(tm + scol, qa + off, ka + off, kIdesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// O_slot (+)= P_slot V (TS: P from TMEM, V block in stage vs as an MN-major
-// operand, N = d).  P of the keys served by softmax column group g (128 /
-// kSplit keys each) sits in the first half of that group's own score
-// columns: keys 16 kk .. 16 kk + 15 at column (kk / G) * 128 / kSplit +
-// (kk % G) * 8 of S_slot, G = 8 / kSplit k-steps per group.
+// O_slot (+)= P_slot V (TS: P from the score buffer at TMEM column pcol, V
+// block in stage vs as an MN-major operand, N = d).  P of the keys served by
+// softmax column group g (128 / kSplit keys each) sits in the first half of
+// that group's own score columns: keys 16 kk .. 16 kk + 15 at column
+// (kk / G) * 128 / kSplit + (kk % G) * 8 of the buffer, G = 8 / kSplit
+// k-steps per group.
 template <int D, int SLOT, bool ACC>
-__device__ __forceinline__ void fwd_issue_pv(uint32_t tm, uint64_t dv, int vs) {
+__device__ __forceinline__ void fwd_issue_pv(uint32_t tm, uint64_t dv, int vs, uint32_t pcol) {
   using C = FwdCfg<D>;
   constexpr uint32_t kIdesc = idesc_bf16(kBM, D, true);
   constexpr int G = (kBN / 16) / kSplit;
@@ -319,8 +326,8 @@ __device__ __forceinline__ void fwd_issue_pv(uint32_t tm, uint64_t dv, int vs) {
 #pragma unroll
   for (int kk = 0; kk < kBN / 16; ++kk) {
     const uint32_t acol = (kk / G) * (kBN / kSplit) + (kk % G) * 8;
-    umma_ts(tm + C::kOCol + SLOT * D, tm + SLOT * 128u + acol, va + ((kk * 16 * 128) >> 4),
-            kIdesc, (ACC || kk > 0) ? 1u : 0u);
+    umma_ts(tm + C::kOCol + SLOT * D, tm + pcol + acol, va + ((kk * 16 * 128) >> 4), kIdesc,
+            (ACC || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -345,10 +352,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* k_empty = k_full + KST;
   uint64_t* v_full = k_empty + KST;
   uint64_t* v_empty = v_full + VST;
-  uint64_t* s_full = v_empty + VST;   // [2]
-  uint64_t* p_full = s_full + 2;      // [2]
-  uint64_t* o_full = p_full + 2;      // [2]
-  uint64_t* mma_done = o_full + 2;
+  // s_full / p_full: scores / P of a slot's block in TMEM, [slot] (d = 128)
+  // or [slot][block parity] (score-buffer pool, d = 64: a slot's softmax
+  // warps may then be a block apart, and two barriers keep the arrivals of
+  // neighbouring blocks apart)
+  uint64_t* s_full = v_empty + VST;   // [4]
+  uint64_t* p_full = s_full + 4;      // [4]
+  uint64_t* o_full = p_full + 4;      // [2]
+  uint64_t* pv_done = o_full + 2;     // [2] (pool) one more P V of the slot done
+  uint64_t* mma_done = pv_done + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -361,12 +373,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
+    // with the score-buffer pool each slot's Q K^T releases its key stage
+    const int k_users = (C::kSBuf == 3 && two) ? 2 : 1;
+    for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], k_users); }
     for (int i = 0; i < VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], 4 * kSplit);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&o_full[i], 1);
+      mbar_init(&pv_done[i], 1);
     }
     mbar_init(mma_done, 1);
     bool bad = false;
@@ -455,14 +472,96 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const uint64_t dk = sdesc_sw128(warp_uniform(smem_k), 16, 1024);
       const uint64_t dv = sdesc_sw128(warp_uniform(smem_v), C::kPanelBytes, 1024);
       bool ok = mbar_wait_warp(q_full, 0, abort_flag) && mbar_wait_warp(&k_full[0], 0, abort_flag);
-      if (ok) {
+      if constexpr (C::kSBuf == 3) {
+        // Pool of three score buffers: the scores of slot s, block j go to
+        // buffer (2 j + s) % 3.  S1(j+1) takes the buffer P0(j) leaves once
+        // P0 V is issued, S0(j+2) the one P1(j) leaves, so each slot's next
+        // scores are computed while its softmax of the current block runs.
+        auto col = [](int j, int s) { return static_cast<uint32_t>(((2 * j + s) % 3) * 128); };
+        if (ok) {
+          tc_fence_after();
+          if (elect_one()) {
+            fwd_issue_s<D, 0>(tm, dq, dk, 0, 0u);
+            umma_commit(&s_full[0]);
+            umma_commit(&k_empty[0]);
+            if (two) {
+              fwd_issue_s<D, 1>(tm, dq, dk, 0, 128u);
+              umma_commit(&s_full[2]);
+              umma_commit(&k_empty[0]);
+            }
+          }
+          __syncwarp();
+          if (n > 1) {
+            ok = mbar_wait_warp(&k_full[1 % KST], (1 / KST) & 1, abort_flag);
+            if (ok) {
+              tc_fence_after();
+              if (elect_one()) {
+                fwd_issue_s<D, 0>(tm, dq, dk, 1 % KST, 256u);
+                umma_commit(&s_full[1]);
+                umma_commit(&k_empty[1 % KST]);
+              }
+              __syncwarp();
+            }
+          }
+        }
+        for (int j = 0; ok && j < n; ++j) {
+          const int vs = j % VST;
+          if (!mbar_wait_warp(&v_full[vs], (j / VST) & 1, abort_flag)) break;
+          if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t pc = col(j, 0);
+            if (j > 0) fwd_issue_pv<D, 0, true>(tm, dv, vs, pc);
+            else fwd_issue_pv<D, 0, false>(tm, dv, vs, pc);
+            umma_commit(&pv_done[0]);
+            if (j == n - 1) umma_commit(&o_full[0]);
+          }
+          __syncwarp();
+          if (two) {
+            if (j + 1 < n) {
+              const int ks = (j + 1) % KST;
+              if (!mbar_wait_warp(&k_full[ks], ((j + 1) / KST) & 1, abort_flag)) break;
+              tc_fence_after();
+              if (elect_one()) {
+                fwd_issue_s<D, 1>(tm, dq, dk, ks, col(j + 1, 1));
+                umma_commit(&s_full[2 + ((j + 1) & 1)]);
+                umma_commit(&k_empty[ks]);
+              }
+              __syncwarp();
+            }
+            if (!mbar_wait_warp(&p_full[2 + (j & 1)], (j >> 1) & 1, abort_flag)) break;
+            tc_fence_after();
+            if (elect_one()) {
+              const uint32_t pc = col(j, 1);
+              if (j > 0) fwd_issue_pv<D, 1, true>(tm, dv, vs, pc);
+              else fwd_issue_pv<D, 1, false>(tm, dv, vs, pc);
+              umma_commit(&pv_done[1]);
+              if (j == n - 1) umma_commit(&o_full[1]);
+            }
+            __syncwarp();
+          }
+          if (j + 2 < n) {
+            const int ks = (j + 2) % KST;
+            if (!mbar_wait_warp(&k_full[ks], ((j + 2) / KST) & 1, abort_flag)) break;
+            tc_fence_after();
+            if (elect_one()) {
+              fwd_issue_s<D, 0>(tm, dq, dk, ks, col(j + 2, 0));
+              umma_commit(&s_full[(j + 2) & 1]);
+              umma_commit(&k_empty[ks]);
+            }
+            __syncwarp();
+          }
+          if (elect_one()) umma_commit(&v_empty[vs]);
+          __syncwarp();
+        }
+      } else if (ok) {
         tc_fence_after();
         if (elect_one()) {
-          fwd_issue_s<D, 0>(tm, dq, dk, 0);
+          fwd_issue_s<D, 0>(tm, dq, dk, 0, 0u);
           umma_commit(&s_full[0]);
           if (two) {
-            fwd_issue_s<D, 1>(tm, dq, dk, 0);
-            umma_commit(&s_full[1]);
+            fwd_issue_s<D, 1>(tm, dq, dk, 0, 128u);
+            umma_commit(&s_full[2]);
           }
           umma_commit(&k_empty[0]);
         }
@@ -477,15 +576,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if (!mbar_wait_warp(&p_full[0], j & 1, abort_flag)) break;
           tc_fence_after();
           if (elect_one()) {
-            if (j > 0) fwd_issue_pv<D, 0, true>(tm, dv, vs);
-            else fwd_issue_pv<D, 0, false>(tm, dv, vs);
+            if (j > 0) fwd_issue_pv<D, 0, true>(tm, dv, vs, 0u);
+            else fwd_issue_pv<D, 0, false>(tm, dv, vs, 0u);
           }
           __syncwarp();
           if (jn < n) {
             if (!mbar_wait_warp(&k_full[ksn], (jn / KST) & 1, abort_flag)) break;
             tc_fence_after();
             if (elect_one()) {
-              fwd_issue_s<D, 0>(tm, dq, dk, ksn);
+              fwd_issue_s<D, 0>(tm, dq, dk, ksn, 0u);
               umma_commit(&s_full[0]);
             }
           } else if (elect_one()) {
@@ -493,14 +592,14 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           }
           __syncwarp();
           if (two) {
-            if (!mbar_wait_warp(&p_full[1], j & 1, abort_flag)) break;
+            if (!mbar_wait_warp(&p_full[2], j & 1, abort_flag)) break;
             tc_fence_after();
             if (elect_one()) {
-              if (j > 0) fwd_issue_pv<D, 1, true>(tm, dv, vs);
-              else fwd_issue_pv<D, 1, false>(tm, dv, vs);
+              if (j > 0) fwd_issue_pv<D, 1, true>(tm, dv, vs, 128u);
+              else fwd_issue_pv<D, 1, false>(tm, dv, vs, 128u);
               if (jn < n) {
-                fwd_issue_s<D, 1>(tm, dq, dk, ksn);
-                umma_commit(&s_full[1]);
+                fwd_issue_s<D, 1>(tm, dq, dk, ksn, 128u);
+                umma_commit(&s_full[2]);
               } else {
                 umma_commit(&o_full[1]);
               }
@@ -537,10 +636,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (!skip && (slot == 0 || two)) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32 + rh * 16) << 16;
       // this warp's 16 lanes; the column half follows from the split offset
-      const uint32_t t_s = tmem + lane_off + (slot ? 128u : 0u);
-      // P over the first half of this thread's own score columns, so no
-      // thread overwrites scores that another has still to read
-      const uint32_t t_p = tmem + lane_off + (slot ? 128u : 0u);
+      // score buffer of this slot (with the d = 64 pool it changes per block)
+      const uint32_t t_s0 = tmem + lane_off;
       const uint32_t t_o = tmem + lane_off + C::kOCol + (slot ? D : 0);
       const float sl2 = p.scale_log2;
       float m_run = -INFINITY;   // running max, log2 units of the scaled scores
@@ -582,8 +679,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         sylo = sylo < 0 ? 0 : (sylo > p.grid_n - swe ? p.grid_n - swe : sylo);
       }
       for (int j = 0; j < n; ++j) {
-        if (!mbar_wait_warp(&s_full[slot], j & 1, abort_flag)) { done = false; break; }
+        // barrier of this slot (and, with the pool, of this block's parity)
+        const int bi = C::kSBuf == 3 ? 2 * slot + (j & 1) : 2 * slot;
+        const uint32_t bph = C::kSBuf == 3 ? (j >> 1) & 1 : j & 1;
+        if (!mbar_wait_warp(&s_full[bi], bph, abort_flag)) { done = false; break; }
         tc_fence_after();
+        const uint32_t scol = C::kSBuf == 3 ? static_cast<uint32_t>(((2 * j + slot) % 3) * 128)
+                                            : (slot ? 128u : 0u);
+        const uint32_t t_s = t_s0 + scol;
+        // P over the first half of this thread's own score columns, so no
+        // thread overwrites scores that another has still to read
+        const uint32_t t_p = t_s;
         float s[kCols];
         // this thread's raw scores of block j, masked (called again by the
         // rare recompute below: the scores stay in TMEM until P is stored)
@@ -729,6 +835,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int cc = 0; cc < kCols / 32; ++cc) tmem_st_half16<kCols>(t_p + cc * 16, pk + cc * 16);
         l_run += lsum;
         if (j > 0 && __any_sync(0xffffffffu, resc)) {
+          if constexpr (C::kSBuf == 3) {
+            // the pool lets this block's scores come before the previous
+            // block's P V: wait until that has landed in O
+            if (!mbar_wait_warp(&pv_done[slot], (j - 1) & 1, abort_flag)) { done = false; break; }
+            tc_fence_after();
+          }
 #pragma unroll
           for (int cc = 0; cc < kOCols / 32; ++cc) {
             uint32_t o[32];
@@ -742,7 +854,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[slot]);
+        if (lane == 0) mbar_arrive(&p_full[bi]);
       }
       if (done && mbar_wait_warp(&o_full[slot], 0, abort_flag)) {
         tc_fence_after();
