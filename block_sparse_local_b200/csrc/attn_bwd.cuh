@@ -9,22 +9,23 @@
 // This file: the preprocessing (D and the log2-domain LSE), the transposed
 // tile lists, and the dK/dV kernel, one 128-row key block per CTA: resident
 // K, V; streams the query blocks whose windows hold that key tile
-// (transposed tile lists), with their -LSE2 and -D.  TMEM: dV [0, d),
-// dK [d, 2d).  The dQ kernel is in attn_bwd_dq.cuh.
-// Each streamed 128-row block is worked on as two 64-row units, alternating
-// between two TMEM score buffers at columns 256 and 384 (S or S^T in 64
-// columns, dP or dP^T in the next 64), so the tensor cores compute the next
-// unit's scores while the elementwise warps turn this unit's scores into P
-// and dS: with one 128-row buffer (the accumulators leave room for no more
-// at d = 128) the score MMAs, the elementwise work and the accumulate MMAs
-// ran strictly one after another.
-// Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (S and dP
-// by SS tcgen05.mma with N = 64, then the accumulators by TS tcgen05.mma with
-// P / dS from TMEM, K = 64), 2-9 elementwise: two warps per TMEM lane
-// quarter, 32 of the unit's 64 columns each.  A warp writes its packed bf16
-// P / dS into the first 16 of its own 32 columns, so no warp overwrites
-// scores another warp still has to read; the accumulate MMAs take the two
-// column groups as two K ranges.
+// (transposed tile lists): Q in a ring of three stages, dO in a ring of two.
+// The dQ kernel is in attn_bwd_dq.cuh.
+// Every MMA has N = 128 (the whole streamed block): an MMA with N = 64
+// costs the tensor cores as long as one with N = 128.  TMEM: dV and dK
+// (fp32), chunk A = S^T of the streamed block, chunk B = dP^T and then the
+// packed P^T and dS^T.  The elementwise warps copy S^T(j) into registers
+// and release chunk A at once, so S(j+1) is computed while they work on
+// block j.  MMA order:
+//   S(0) dP(0) S(1) | dV(0) dK(0) dP(1) S(2) | dV(1) dK(1) dP(2) S(3) | ...
+// Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (scores
+// by SS tcgen05.mma, the accumulators by TS tcgen05.mma with P^T / dS^T from
+// TMEM), 2-17 elementwise: four warps per TMEM lane quarter, 32 of the 128
+// streamed rows (score columns) each.  A warp writes its packed bf16 P^T
+// and dS^T over its own 32 columns of chunk B (P^T in the first 16, dS^T in
+// the last 16), so no warp overwrites scores another warp still has to
+// read; the accumulate MMAs take two K steps of 16 rows from each warp's
+// columns.
 #pragma once
 
 #include <type_traits>
@@ -34,7 +35,14 @@
 
 namespace sta {
 
-constexpr int kBwdThreads = 320;
+constexpr int kDkvEwWarps = 16;         // dK/dV kernel: elementwise warps
+constexpr int kDkvThreads = 64 + 32 * kDkvEwWarps;
+// Exponentials of the dK/dV kernel on the FMA pipe: this many of every 8
+// column pairs (the rest on the ex2 unit).
+#ifndef STA_DKV_EXP2_FMA_PAIRS
+#define STA_DKV_EXP2_FMA_PAIRS 2
+#endif
+constexpr int kDkvExp2FmaPairs = STA_DKV_EXP2_FMA_PAIRS;
 
 struct BwdParams {
   const WorkItem* items;
@@ -62,13 +70,15 @@ struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kBlockBytes = 128 * D * 2;
-  static constexpr int kStages = 2;
-  static constexpr int kResA = 0;                                  // K (dKV) / Q (dQ)
-  static constexpr int kResB = kResA + kBlockBytes;                // V (dKV) / dO (dQ)
-  static constexpr int kStream = kResB + kBlockBytes;              // per stage: 2 blocks + vec
-  static constexpr int kStageBytes = 2 * kBlockBytes + 1024;
-  static constexpr int kBarOff = kStream + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr int kQStages = 3;
+  static constexpr int kDoStages = 2;
+  static constexpr int kResK = 0;
+  static constexpr int kResV = kResK + kBlockBytes;
+  static constexpr int kQRing = kResV + kBlockBytes;
+  static constexpr int kDoRing = kQRing + kQStages * kBlockBytes;
+  static constexpr int kBarOff = kDoRing + kDoStages * kBlockBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;   // + 1024-byte alignment
+  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
 
 // One warp per two rows: D[row] = sum_c dO[row,c] * O[row,c] (fp32) and the
@@ -138,18 +148,18 @@ __global__ void __launch_bounds__(128) kv_tile_list_transposed_kernel(
   for (int i = n; i < g.max_k; ++i) out[i] = -1;
 }
 
-// TMEM columns: the accumulators (dV at 0 and dK at d, or dQ at 0), then two
-// score buffers of one 64-row unit each: S (or S^T) in 64 columns, dP (or
-// dP^T) in the next 64.
-constexpr uint32_t kBwdBufCol = 256;
+// TMEM columns of the two 128-column chunks (the accumulators: dV at 0, dK
+// at d).
+constexpr uint32_t kDkvColA = 256;
+constexpr uint32_t kDkvColB = 384;
 
-// Scores of one 64-row unit of a streamed block: D = A B^T over d (SS, both
-// K-major, M = 128 resident rows, N = 64).  a: resident block descriptor, b:
-// descriptor of the unit's first row (address field already offset).
+// Scores of a streamed block: D = A B^T over d (SS, both K-major, M = 128
+// resident rows, N = 128 streamed rows).  a: resident block descriptor, b:
+// descriptor of the streamed block (address field already offset).
 template <int D>
-__device__ __forceinline__ void bwd_issue_ss_unit(uint32_t d_tmem, uint64_t a, uint64_t b) {
+__device__ __forceinline__ void bwd_issue_scores(uint32_t d_tmem, uint64_t a, uint64_t b) {
   using C = BwdCfg<D>;
-  constexpr uint32_t kIdS = idesc_bf16(128, 64, false);
+  constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = ((kk >> 2) * C::kPanelBytes + (kk & 3) * 32) >> 4;
@@ -157,39 +167,43 @@ __device__ __forceinline__ void bwd_issue_ss_unit(uint32_t d_tmem, uint64_t a, u
   }
 }
 
-// acc (+)= A B over one 64-row unit: A packed bf16 in TMEM, K = 64 rows of
-// the unit, columns [a, a+16) (rows 0..31, first column group) and
-// [a+32, a+48) (rows 32..63, second group); B the unit's rows of a streamed
-// block as an MN-major operand (N = d).  ACC: accumulate flag of the first
-// k-step.
+// acc (+)= A B over a streamed block: A packed bf16 in TMEM, K = the 128
+// streamed rows in four groups of 32 (rows 32 g .. 32 g + 31 packed into
+// columns [a + 32 g, a + 32 g + 16)); B the streamed block as an MN-major
+// operand (N = d).  ACC: accumulate flag of the first k-step.
 template <int D, bool ACC>
-__device__ __forceinline__ void bwd_issue_ts_unit(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
+__device__ __forceinline__ void bwd_issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
   constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
+  for (int kk = 0; kk < 8; ++kk) {
     const uint32_t acol = (kk >> 1) * 32 + (kk & 1) * 8;
     umma_ts(d_tmem, a_tmem + acol, b + ((kk * 16 * 128) >> 4), kIdAcc, (ACC || kk > 0) ? 1u : 0u);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tmap_q,
                     const __grid_constant__ CUtensorMap tmap_k,
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int ST = C::kStages;
+  constexpr int QS = C::kQStages;
+  constexpr int OS = C::kDoStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* res_full = bars;
-  uint64_t* full = res_full + 1;         // [ST]
-  uint64_t* empty = full + ST;           // [ST]
-  uint64_t* s_full = empty + ST;         // [2] per score buffer
-  uint64_t* p_full = s_full + 2;         // [2]
-  uint64_t* acc_full = p_full + 2;
+  uint64_t* q_full = res_full + 1;       // [QS]
+  uint64_t* q_empty = q_full + QS;       // [QS]
+  uint64_t* do_full = q_empty + QS;      // [OS]
+  uint64_t* do_empty = do_full + OS;     // [OS]
+  uint64_t* s_full = do_empty + OS;      // S^T of the next block in chunk A
+  uint64_t* s_free = s_full + 1;         // every elementwise warp holds S^T: chunk A free
+  uint64_t* dp_full = s_free + 1;        // dP^T in chunk B
+  uint64_t* pd_full = dp_full + 1;       // packed P^T and dS^T written
+  uint64_t* acc_full = pd_full + 1;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -202,7 +216,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                               item.kv_base >= 0 && item.kv_base < p.dbg_rows &&
                               item.list >= 0 && item.list < p.dbg_lists) &&
                        dbg_ok(p.counts[item.list] >= 0 && p.counts[item.list] <= p.max_k);
-  // stream: key blocks of the query block (dQ) or query blocks of the key block (dK/dV)
+  // streamed query blocks of the key block
   const int cnt = item_ok ? p.counts[item.list] : 0;
   const int* ids = p.ids + static_cast<size_t>(item_ok ? item.list : 0) * p.max_k;
   const int nvid = (cnt - p.text_sentinel) * p.tile_blocks;
@@ -217,11 +231,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(res_full, 1);
-    for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 8);
-    }
+    for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
+    for (int i = 0; i < OS; ++i) { mbar_init(&do_full[i], 1); mbar_init(&do_empty[i], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kDkvEwWarps);
+    mbar_init(dp_full, 1);
+    mbar_init(pd_full, kDkvEwWarps);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
@@ -239,132 +254,125 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const bool skip = *abort_flag != 0;
-  const uint32_t s_res_a = smem_u32(smem + C::kResA);
-  const uint32_t s_res_b = smem_u32(smem + C::kResB);
-  const uint32_t s_stream = smem_u32(smem + C::kStream);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // A thread's TMA loads complete one after another, so every operand
-    // panel has its own lane: lanes 0 .. kPanels-1 the panels of the first
-    // streamed operand (Q for dK/dV, K for dQ) and of the resident K / Q,
-    // lanes kPanels .. 2 kPanels-1 those of the second (dO / V, resident
-    // V / dO), lane 2 kPanels the two 512-byte LSE / D copies (dK/dV).  Lane
-    // 0 posts the expected bytes of every stage.
+    // panel has its own lane: lanes 0 .. kPanels-1 the panels of resident K
+    // and of the streamed Q blocks, lanes kPanels .. 2 kPanels-1 those of
+    // resident V and of the streamed dO blocks.  The first lane of each
+    // operand posts the expected bytes.
     constexpr int kPanels = C::kPanels;
-    constexpr int kLanes = 2 * kPanels + 1;
+    constexpr int kLanes = 2 * kPanels;
     if (lane < kLanes && !skip) {
       const uint64_t pol = policy_evict_last();
-      const int row0 = item.q0;   // the resident block
-      const bool is_b = lane >= kPanels && lane < 2 * kPanels;
-      const bool is_vec = lane == 2 * kPanels;
+      const bool is_do = lane >= kPanels;
       const int pn = lane % kPanels;
       if (lane == 0) mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
-      if (!is_vec) {
-        const CUtensorMap* mres = is_b ? &tmap_v : &tmap_k;
-        tma_load_2d_hint(smem + (is_b ? C::kResB : C::kResA) + pn * C::kPanelBytes, mres,
-                         res_full, pn * 64, row0, pol);
-      }
-      const CUtensorMap* mstr = is_b ? &tmap_do : &tmap_q;
+      tma_load_2d_hint(smem + (is_do ? C::kResV : C::kResK) + pn * C::kPanelBytes,
+                       is_do ? &tmap_v : &tmap_k, res_full, pn * 64, item.q0, pol);
+      const CUtensorMap* mstr = is_do ? &tmap_do : &tmap_q;
+      const int ns = is_do ? OS : QS;
+      uint64_t* fullb = is_do ? do_full : q_full;
+      uint64_t* emptyb = is_do ? do_empty : q_empty;
+      uint8_t* ring = smem + (is_do ? C::kDoRing : C::kQRing);
       for (int j = 0; j < n; ++j) {
-        const int st = j % ST;
-        if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
+        const int st = j % ns;
+        if (j >= ns && !mbar_wait(&emptyb[st], ((j / ns) - 1) & 1, abort_flag)) break;
         const int row = stream_row(j);
         if (!dbg_ok(row >= 0 && row + 128 <= p.dbg_rows)) {
           *abort_flag = 1;
           break;
         }
-        uint8_t* base = smem + C::kStream + st * C::kStageBytes;
-        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + 1024);
-        if (!is_vec) {
-          tma_load_2d_hint(base + (is_b ? C::kBlockBytes : 0) + pn * C::kPanelBytes, mstr,
-                           &full[st], pn * 64, row, pol);
-        } else {
-          // the streamed query block's -lse2 and -D (2 x 512 bytes)
-          asm volatile(
-              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
-              "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes)),
-              "l"(reinterpret_cast<uint64_t>(p.neg_lse2 + row)), "r"(smem_u32(&full[st]))
-              : "memory");
-          asm volatile(
-              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
-              "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes + 512)),
-              "l"(reinterpret_cast<uint64_t>(p.neg_delta + row)), "r"(smem_u32(&full[st]))
-              : "memory");
+        if (pn == 0) mbar_arrive_expect_tx(&fullb[st], C::kBlockBytes);
+        tma_load_2d_hint(ring + st * C::kBlockBytes + pn * C::kPanelBytes, mstr, &fullb[st],
+                         pn * 64, row, pol);
+        // the elementwise warps read this block's -lse2 and -D with plain
+        // loads: bring their 2 x 4 lines into L1 ahead of them
+        if (lane == 0) {
+#pragma unroll
+          for (int l = 0; l < 4; ++l) {
+            prefetch_l1(p.neg_lse2 + row + 32 * l);
+            prefetch_l1(p.neg_delta + row + 32 * l);
+          }
         }
       }
       __syncwarp((1u << kLanes) - 1u);
       // Leave no copy in flight: wait for the last load of every stage.
       if (lane == 0) {
         mbar_wait_drain(res_full, 0);
-        for (int st = 0; st < ST && st < n; ++st) {
-          const int last = st + ((n - 1 - st) / ST) * ST;
-          mbar_wait_drain(&full[st], (last / ST) & 1);
+        for (int st = 0; st < QS && st < n; ++st) {
+          const int last = st + ((n - 1 - st) / QS) * QS;
+          mbar_wait_drain(&q_full[st], (last / QS) & 1);
+        }
+        for (int st = 0; st < OS && st < n; ++st) {
+          const int last = st + ((n - 1 - st) / OS) * OS;
+          mbar_wait_drain(&do_full[st], (last / OS) & 1);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Whole warp waits, one elected lane (always the same) issues; every MMA
-    // operand is warp-uniform and every accumulate flag a constant.
+    // operand is warp-uniform and every accumulate flag a constant.  S(j+2)
+    // overwrites chunk A once every elementwise warp holds S(j+1) in
+    // registers; dP(j+1) overwrites chunk B after dV(j) and dK(j), the last
+    // readers of P(j) and dS(j): tcgen05 MMAs of one thread execute in issue
+    // order.
     if (!skip) {
       const uint32_t tm = warp_uniform(tmem);
-      const uint64_t d_res_a = sdesc_sw128(warp_uniform(s_res_a), 16, 1024);
-      const uint64_t d_res_b = sdesc_sw128(warp_uniform(s_res_b), 16, 1024);
-      const uint64_t d_str_k = sdesc_sw128(warp_uniform(s_stream), 16, 1024);
-      const uint64_t d_str_mn = sdesc_sw128(warp_uniform(s_stream), C::kPanelBytes, 1024);
-      // Units u = 0 .. 2n-1: the two 64-row halves of streamed block u / 2,
-      // in score buffer u % 2.  Scores of unit u + 2 go into the buffer that
-      // the accumulate MMAs of unit u read, issued right after them (tcgen05
-      // MMAs of one thread execute in issue order), so the scores of the next
-      // unit are computed while the elementwise warps work on this one.
-      const int U = 2 * n;
-      auto issue_scores = [&](int u) {
-        const int st = (u >> 1) % ST;
-        const uint32_t so = (static_cast<uint32_t>(st) * C::kStageBytes + (u & 1) * 64 * 128) >> 4;
-        const uint32_t sb = so + (C::kBlockBytes >> 4);
-        const uint32_t buf = tm + kBwdBufCol + (u & 1) * 128;
+      const uint64_t d_res_k = sdesc_sw128(warp_uniform(smem_u32(smem + C::kResK)), 16, 1024);
+      const uint64_t d_res_v = sdesc_sw128(warp_uniform(smem_u32(smem + C::kResV)), 16, 1024);
+      const uint32_t s_q = warp_uniform(smem_u32(smem + C::kQRing));
+      const uint32_t s_do = warp_uniform(smem_u32(smem + C::kDoRing));
+      const uint64_t d_q_k = sdesc_sw128(s_q, 16, 1024);
+      const uint64_t d_q_mn = sdesc_sw128(s_q, C::kPanelBytes, 1024);
+      const uint64_t d_do_k = sdesc_sw128(s_do, 16, 1024);
+      const uint64_t d_do_mn = sdesc_sw128(s_do, C::kPanelBytes, 1024);
+      auto q_off = [](int j) { return static_cast<uint32_t>((j % QS) * C::kBlockBytes) >> 4; };
+      auto do_off = [](int j) { return static_cast<uint32_t>((j % OS) * C::kBlockBytes) >> 4; };
+      // S(j) = K Q_j^T into chunk A once Q_j has landed
+      auto issue_s = [&](int j) -> bool {
+        if (!mbar_wait_warp(&q_full[j % QS], (j / QS) & 1, abort_flag)) return false;
+        tc_fence_after();
         if (elect_one()) {
-          bwd_issue_ss_unit<D>(buf, d_res_a, d_str_k + so);        // S^T = K Q^T  |  S = Q K^T
-          bwd_issue_ss_unit<D>(buf + 64, d_res_b, d_str_k + sb);   // dP^T = V dO^T |  dP = dO V^T
-          umma_commit(&s_full[u & 1]);
+          bwd_issue_scores<D>(tm + kDkvColA, d_res_k, d_q_k + q_off(j));
+          umma_commit(s_full);
         }
         __syncwarp();
+        return true;
       };
-      bool ok = mbar_wait_warp(res_full, 0, abort_flag) && mbar_wait_warp(&full[0], 0, abort_flag);
-      if (ok) {
+      // dP(j) = V dO_j^T into chunk B once dO_j has landed
+      auto issue_dp = [&](int j) -> bool {
+        if (!mbar_wait_warp(&do_full[j % OS], (j / OS) & 1, abort_flag)) return false;
         tc_fence_after();
-        issue_scores(0);
-        issue_scores(1);
-      }
-      for (int u = 0; ok && u < U; ++u) {
-        const int st = (u >> 1) % ST;
-        if (!mbar_wait_warp(&p_full[u & 1], (u >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t so = (static_cast<uint32_t>(st) * C::kStageBytes + (u & 1) * 64 * 128) >> 4;
-        const uint32_t sb = so + (C::kBlockBytes >> 4);
-        const uint32_t buf = tm + kBwdBufCol + (u & 1) * 128;
         if (elect_one()) {
-          if (u > 0) {
-            bwd_issue_ts_unit<D, true>(tm, buf, d_str_mn + sb);           // dV += P^T dO
-            bwd_issue_ts_unit<D, true>(tm + D, buf + 64, d_str_mn + so);  // dK += dS^T Q
-          } else {
-            bwd_issue_ts_unit<D, false>(tm, buf, d_str_mn + sb);
-            bwd_issue_ts_unit<D, false>(tm + D, buf + 64, d_str_mn + so);
-          }
-          if (u & 1) umma_commit(&empty[st]);   // both units of the stage consumed
-          if (u == U - 1) umma_commit(acc_full);
+          bwd_issue_scores<D>(tm + kDkvColB, d_res_v, d_do_k + do_off(j));
+          umma_commit(dp_full);
         }
         __syncwarp();
-        const int un = u + 2;
-        if (un < U) {
-          if ((un & 1) == 0) {
-            const int jn = un >> 1;
-            if (!mbar_wait_warp(&full[jn % ST], (jn / ST) & 1, abort_flag)) break;
-            tc_fence_after();
+        return true;
+      };
+      bool ok = mbar_wait_warp(res_full, 0, abort_flag) && issue_s(0) && issue_dp(0);
+      if (ok && n > 1) ok = mbar_wait_warp(s_free, 0, abort_flag) && issue_s(1);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait_warp(pd_full, j & 1, abort_flag)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          if (j > 0) {
+            bwd_issue_acc<D, true>(tm, tm + kDkvColB, d_do_mn + do_off(j));           // dV += P^T dO
+            bwd_issue_acc<D, true>(tm + D, tm + kDkvColB + 16, d_q_mn + q_off(j));    // dK += dS^T Q
+          } else {
+            bwd_issue_acc<D, false>(tm, tm + kDkvColB, d_do_mn + do_off(j));
+            bwd_issue_acc<D, false>(tm + D, tm + kDkvColB + 16, d_q_mn + q_off(j));
           }
-          issue_scores(un);
+          umma_commit(&do_empty[j % OS]);   // dP(j) and dV(j) were the readers of dO_j
+          umma_commit(&q_empty[j % QS]);    // S(j) and dK(j) those of Q_j
+          if (j == n - 1) umma_commit(acc_full);
         }
+        __syncwarp();
+        if (j + 1 < n && !issue_dp(j + 1)) break;
+        if (j + 2 < n && !(mbar_wait_warp(s_free, (j + 1) & 1, abort_flag) && issue_s(j + 2))) break;
       }
       if (elect_one()) umma_commit(mma_done);
       __syncwarp();
@@ -373,112 +381,121 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ elementwise
     const int ks = warp - 2;
-    const int half = ks >> 2;
-    const int sub = warp & 3;
+    const int cg = ks >> 2;                             // 32-column group of the scores
+    const int sub = warp & 3;                           // TMEM lane quarter
     const int r = sub * 32 + lane;                      // row of the resident block
     const int my_row = item.q0 + r;
     if (!skip) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const float sl2 = p.scale_log2;
+      const uint32_t t_a = tmem + lane_off + kDkvColA + cg * 32;
+      const uint32_t t_b = tmem + lane_off + kDkvColB + cg * 32;
+      const float2 sl2v = make_float2(p.scale_log2, p.scale_log2);
       // whether this key row is valid (padded text keys are not)
       bool row_valid = true;
       {
         const int off = my_row - item.kv_base;
         if (off >= p.L_v) row_valid = (off - p.L_v) < p.text_len;
       }
+      // padded text key rows give zero P and dS
+      const bool masked = !__all_sync(0xffffffffu, row_valid);
       bool done = true;
-      for (int u = 0; u < 2 * n; ++u) {
-        const int j = u >> 1;           // streamed block
-        const int hu = u & 1;           // its 64-row half, and the score buffer
-        const int st = j % ST;
-        if (!mbar_wait_warp(&s_full[hu], j & 1, abort_flag)) { done = false; break; }
-        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
-        tc_fence_after();
-        const uint32_t t_s = tmem + lane_off + kBwdBufCol + hu * 128 + half * 32;
-        const uint32_t t_dp = t_s + 64;
-        uint32_t sr[32], dr[32];
-        STA_TMEM_LD32(t_s, sr);
-        STA_TMEM_LD32(t_dp, dr);
-        tmem_wait_ld();
-        // padded text key rows give zero P and dS
-        const bool masked = !__all_sync(0xffffffffu, row_valid);
-        // -lse2 and -D of this warp's 32 streamed rows, 16-byte aligned in
-        // the stage
-        const float4* nl4p = reinterpret_cast<const float4*>(
-            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + hu * 16 + half * 8;
-        const float4* nd4p = nl4p + 32;
-        uint32_t pk_p[16], pk_ds[16];
-        // P = exp2(S sl2 - lse2) and dS = P (dP - D), two columns at a time
-        // (packed f32x2 FMA / ADD / MUL; a fixed share of the exponentials on
-        // the FMA pipe), packed to bf16 as they come
-        auto elementwise = [&](auto with_mask) {
-          const float2 sl2v = make_float2(sl2, sl2);
+      for (int j = 0; j < n; ++j) {
+        // -lse2 and -D of this warp's 32 streamed rows (the same address in
+        // every lane: one L1 transaction per load)
+        const int q_row = stream_row(j) + cg * 32;
+        const float4* nl4p = reinterpret_cast<const float4*>(p.neg_lse2 + q_row);
+        const float4* nd4p = reinterpret_cast<const float4*>(p.neg_delta + q_row);
+        float4 nl4v[8];
 #pragma unroll
-          for (int e4 = 0; e4 < 8; ++e4) {
-            const float4 nl4 = nl4p[e4];
-            const float4 nd4 = nd4p[e4];
+        for (int e4 = 0; e4 < 8; ++e4) nl4v[e4] = __ldg(nl4p + e4);
+        if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        uint32_t sr[32];
+        STA_TMEM_LD32(t_a, sr);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(s_free);
+        // P = exp2(S sl2 - lse2), two columns at a time (packed f32x2 FMA; a
+        // fixed share of the exponentials on the FMA pipe), kept in fp32 for
+        // dS and packed to bf16 as they come
+        float2 pr[16];
+        uint32_t pk_p[16];
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 nl4 = nl4v[e4];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int e = 2 * e4 + h2;       // column pair
+            const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2v, nl);
+            float2 pe;
+            if (exp2_on_fma_of<kDkvExp2FmaPairs>(e)) {   // resolved at compile time
+              pe = exp2_fma2(x);
+            } else {
+              pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+            }
+            if (masked && !row_valid) pe = make_float2(0.f, 0.f);
+            pr[e] = pe;
+            pk_p[e] = pack_bf16x2(pe.x, pe.y);
+          }
+        }
+        // dS = P (dP - D)
+        if (!mbar_wait_warp(dp_full, j & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        // (dP^T in two halves of 16 columns, to stay within the registers of
+        // 18 warps)
+        uint32_t pk_ds[16];
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t dr[16];
+          STA_TMEM_LD16(t_b + hf * 16, dr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 nd4 = __ldg(nd4p + hf * 4 + e4);
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-              const int e = 2 * e4 + h2;       // column pair
-              const int c = 2 * e;
-              const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+              const int c = 2 * e4 + h2;     // column pair within the half
+              const int e = hf * 8 + c;
               const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-              const float2 x = __ffma2_rn(
-                  make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, nl);
-              float2 pr;
-              if (exp2_on_fma(e)) {   // resolved at compile time (unrolled)
-                pr = exp2_fma2(x);
-              } else {
-                pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-              }
-              if constexpr (decltype(with_mask)::value) {
-                if (!row_valid) pr = make_float2(0.f, 0.f);
-              }
               const float2 ds = __fmul2_rn(
-                  pr, __fadd2_rn(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])),
-                                 nd));
-              pk_p[e] = pack_bf16x2(pr.x, pr.y);
+                  pr[e], __fadd2_rn(make_float2(__uint_as_float(dr[2 * c]),
+                                                __uint_as_float(dr[2 * c + 1])), nd));
               pk_ds[e] = pack_bf16x2(ds.x, ds.y);
             }
           }
-        };
-        if (masked) {
-          elementwise(std::true_type{});
-        } else {
-          elementwise(std::false_type{});
         }
-        // packed bf16 over the first 16 of this warp's own 32 columns, so no
-        // warp overwrites scores another warp still has to read
-        STA_TMEM_ST16(t_s, pk_p);     // P^T
-        STA_TMEM_ST16(t_dp, pk_ds);   // dS^T
+        STA_TMEM_ST16(t_b, pk_p);          // P^T
+        STA_TMEM_ST16(t_b + 16, pk_ds);    // dS^T
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[hu]);
+        if (lane == 0) mbar_arrive(pd_full);
       }
       if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
         tc_fence_after();
-        constexpr int kHalfCols = D / 2;
+        // each warp writes D / 4 columns of its rows of dV and of dK
+        constexpr int kQCols = D / 4;
         for (int a = 0; a < 2; ++a) {
           // a = 0 -> dV (unscaled), a = 1 -> dK (scaled)
-          const uint32_t t_acc = tmem + lane_off + (a == 1 ? D : 0) + half * kHalfCols;
+          const uint32_t t_acc = tmem + lane_off + (a == 1 ? D : 0) + cg * kQCols;
           const float sc = a == 0 ? 1.f : p.scale;
           __nv_bfloat16* dstp = a == 0 ? p.out_b : p.out_a;
           uint4* dst = reinterpret_cast<uint4*>(dstp + static_cast<size_t>(my_row) * D +
-                                                half * kHalfCols);
+                                                cg * kQCols);
 #pragma unroll
-          for (int cc = 0; cc < kHalfCols / 32; ++cc) {
-            uint32_t o[32];
-            STA_TMEM_LD32(t_acc + cc * 32, o);
+          for (int cc = 0; cc < kQCols / 16; ++cc) {
+            uint32_t o[16];
+            STA_TMEM_LD16(t_acc + cc * 16, o);
             tmem_wait_ld();
-            uint32_t pk[16];
+            uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e)
+            for (int e = 0; e < 8; ++e)
               pk[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * sc, __uint_as_float(o[2 * e + 1]) * sc);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[cc * 4 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2],
-                                            pk[4 * v4 + 3]);
+            dst[cc * 2] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[cc * 2 + 1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
           }
         }
       }

@@ -7,17 +7,21 @@
 // three stages (released after dQ += dS K reads it) and V in two (released
 // right after the dP MMA, its only reader).
 //
-// TMEM: the dQ accumulator in columns [0, 128); S(j) of key block j alternates
-// between [128, 256) and [384, 512); dP(j) in [256, 384).  The elementwise
-// warps first copy S(j) and dP(j) into registers (after which [256, 384) may
-// take dP(j+1)) and then write their packed bf16 dS(j) over their own columns
-// of S(j), which dQ += dS K reads.  So the tensor cores compute S(j+1) and
-// dP(j+1) while the elementwise warps work on block j, and the accumulate
-// MMA of block j follows them.
+// TMEM: the dQ accumulator in columns [0, 128); the resident Q and dO,
+// packed bf16, in [128, 192) and [192, 256) (copied from shared memory by
+// tcgen05.cp), so that S = Q K^T and dP = dO V^T are TS MMAs that read only
+// K and V from shared memory (SS MMAs reading both operands there ran at two
+// thirds of the tensor rate: shared-memory bandwidth); S(j) in [256, 384),
+// dP(j) and then the packed dS(j) in [384, 512).  The elementwise warps copy
+// S(j) into registers and release its columns at once, so S(j+1) is computed
+// while they work on block j.  MMA order:
+//   S(0) dP(0) S(1) | acc(0) dP(1) S(2) | acc(1) dP(2) S(3) | ...
 // Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (the whole
 // warp waits, one elected lane issues; warp-uniform operands, constant
-// accumulate flags), 2-9 elementwise: two warps per TMEM lane quarter, 64 of
-// the 128 key columns each.
+// accumulate flags), 2-17 elementwise: four warps per TMEM lane quarter, 32
+// of the 128 key columns each (the dS work of block j+1 sits on the loop
+// acc(j) -> dP(j+1) -> dS(j+1), so it is spread over as many warps as the
+// registers allow).
 #pragma once
 
 #include <type_traits>
@@ -26,6 +30,9 @@
 #include "attn_bwd.cuh"
 
 namespace sta {
+
+constexpr int kDqEwWarps = 16;          // dQ kernel: elementwise warps
+constexpr int kDqThreads = 64 + 32 * kDqEwWarps;
 
 template <int D>
 struct BwdDqCfg {
@@ -43,37 +50,50 @@ struct BwdDqCfg {
   static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
 
-// TMEM column of S(j); dP always at 256.
-__device__ __forceinline__ uint32_t bwd_dq_s_col(int j) { return (j & 1) ? 384u : 128u; }
-constexpr uint32_t kBwdDqDpCol = 256;
+constexpr uint32_t kBwdDqColQ = 128;    // resident Q, packed bf16
+constexpr uint32_t kBwdDqColDo = 192;   // resident dO, packed bf16
+constexpr uint32_t kBwdDqColS = 256;    // S(j)
+constexpr uint32_t kBwdDqColDp = 384;   // dP(j), then the packed dS(j)
 
-// D = A B^T over d (SS, both K-major, 128 x 128).  a, b: block descriptors
-// (address field already offset).
+// Descriptor offset (16-byte units) of k-step kk of a K-major block.
 template <int D>
-__device__ __forceinline__ void bwd_dq_issue_ss(uint32_t d_tmem, uint64_t a, uint64_t b) {
-  constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = ((kk >> 2) * BwdDqCfg<D>::kPanelBytes + (kk & 3) * 32) >> 4;
-    umma_ss(d_tmem, a + off, b + off, kIdS, kk > 0 ? 1u : 0u);
-  }
+__device__ __forceinline__ uint32_t bwd_dq_kstep_off(int kk) {
+  return static_cast<uint32_t>((kk >> 2) * BwdDqCfg<D>::kPanelBytes + (kk & 3) * 32) >> 4;
 }
 
-// dQ (+)= dS K: dS packed bf16 in TMEM (keys 0..63 in columns [a, a+32) of
-// the first column group, keys 64..127 in [a+64, a+96) of the second), K an
-// MN-major block (N = d).  ACC: accumulate flag of the first k-step.
+// Copy a resident block (K-major in shared memory) into TMEM as a packed
+// bf16 A operand: k-step kk into columns [t + 8 kk, t + 8 kk + 8).
+template <int D>
+__device__ __forceinline__ void bwd_dq_copy_res(uint32_t t, uint64_t desc) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) tmem_cp_128x256b(t + kk * 8, desc + bwd_dq_kstep_off<D>(kk));
+}
+
+// D = A B^T over d (TS: A the resident block in TMEM, B a streamed K-major
+// block in shared memory; 128 x 128).
+template <int D>
+__device__ __forceinline__ void bwd_dq_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
+  constexpr uint32_t kIdS = idesc_bf16(128, 128, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk)
+    umma_ts(d_tmem, a_tmem + kk * 8, b + bwd_dq_kstep_off<D>(kk), kIdS, kk > 0 ? 1u : 0u);
+}
+
+// dQ (+)= dS K: dS packed bf16 in TMEM (keys 32 g .. 32 g + 31 in columns
+// [a + 32 g, a + 32 g + 16)), K an MN-major block (N = d).  ACC: accumulate
+// flag of the first k-step.
 template <int D, bool ACC>
 __device__ __forceinline__ void bwd_dq_issue_acc(uint32_t d_tmem, uint32_t a_tmem, uint64_t b) {
   constexpr uint32_t kIdAcc = idesc_bf16(128, D, true);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const uint32_t acol = (kk >> 2) * 64 + (kk & 3) * 8;
+    const uint32_t acol = (kk >> 1) * 32 + (kk & 1) * 8;
     umma_ts(d_tmem, a_tmem + acol, b + ((kk * 16 * 128) >> 4), kIdAcc, (ACC || kk > 0) ? 1u : 0u);
   }
 }
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmap_q,
                        const __grid_constant__ CUtensorMap tmap_k,
                        const __grid_constant__ CUtensorMap tmap_v,
@@ -90,10 +110,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* k_empty = k_full + KST;      // [KST]
   uint64_t* v_full = k_empty + KST;      // [VST]
   uint64_t* v_empty = v_full + VST;      // [VST]
-  uint64_t* s_full = v_empty + VST;      // S(j) and dP(j) computed
-  uint64_t* d_free = s_full + 1;         // the elementwise warps have loaded S(j), dP(j)
-  uint64_t* p_full = d_free + 1;         // [2 by block parity] dS(j) stored
-  uint64_t* acc_full = p_full + 2;
+  uint64_t* s_full = v_empty + VST;      // S(j) computed
+  uint64_t* s_free = s_full + 1;         // every elementwise warp holds S(j): columns free
+  uint64_t* dp_full = s_free + 1;        // dP(j) computed
+  uint64_t* ds_full = dp_full + 1;       // packed dS(j) written
+  uint64_t* acc_full = ds_full + 1;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -124,8 +145,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int i = 0; i < KST; ++i) { mbar_init(&k_full[i], 1); mbar_init(&k_empty[i], 1); }
     for (int i = 0; i < VST; ++i) { mbar_init(&v_full[i], 1); mbar_init(&v_empty[i], 1); }
     mbar_init(s_full, 1);
-    mbar_init(d_free, 8);
-    for (int i = 0; i < 2; ++i) mbar_init(&p_full[i], 8);
+    mbar_init(s_free, kDqEwWarps);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, kDqEwWarps);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
@@ -191,10 +213,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per key block j: S(j+1) into the S column block that the accumulate
-    // MMA of block j-1 read (issued before it; tcgen05 MMAs of one thread
-    // execute in issue order), dP(j+1) once the elementwise warps have
-    // loaded dP(j), then dQ += dS(j) K(j).
+    // S(j+2) overwrites S's columns once every elementwise warp holds S(j+1)
+    // in registers; dP(j+1) overwrites the packed dS(j) after acc(j), its
+    // reader (tcgen05 ops of one thread execute in issue order).
     if (!skip) {
       const uint32_t tm = warp_uniform(tmem);
       const uint64_t d_q = sdesc_sw128(warp_uniform(smem_u32(smem + C::kQOff)), 16, 1024);
@@ -203,53 +224,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t d_kmn =
           sdesc_sw128(warp_uniform(smem_u32(smem + C::kKOff)), C::kPanelBytes, 1024);
       const uint64_t d_v = sdesc_sw128(warp_uniform(smem_u32(smem + C::kVOff)), 16, 1024);
-      auto issue_s = [&](int j) {       // S = Q K^T
+      auto issue_s = [&](int j) -> bool {      // S = Q K^T once K(j) has landed
+        if (!mbar_wait_warp(&k_full[j % KST], (j / KST) & 1, abort_flag)) return false;
+        tc_fence_after();
         const uint32_t off = (static_cast<uint32_t>(j % KST) * C::kBlockBytes) >> 4;
-        if (elect_one()) bwd_dq_issue_ss<D>(tm + bwd_dq_s_col(j), d_q, d_k + off);
+        if (elect_one()) {
+          bwd_dq_issue_ts<D>(tm + kBwdDqColS, tm + kBwdDqColQ, d_k + off);
+          umma_commit(s_full);
+        }
         __syncwarp();
+        return true;
       };
-      auto issue_dp = [&](int j) {      // dP = dO V^T; V's stage is free once it is done
+      auto issue_dp = [&](int j) -> bool {     // dP = dO V^T; V's only reader
         const int vs = j % VST;
+        if (!mbar_wait_warp(&v_full[vs], (j / VST) & 1, abort_flag)) return false;
+        tc_fence_after();
         const uint32_t off = (static_cast<uint32_t>(vs) * C::kBlockBytes) >> 4;
         if (elect_one()) {
-          bwd_dq_issue_ss<D>(tm + kBwdDqDpCol, d_do, d_v + off);
-          umma_commit(s_full);
+          bwd_dq_issue_ts<D>(tm + kBwdDqColDp, tm + kBwdDqColDo, d_v + off);
+          umma_commit(dp_full);
           umma_commit(&v_empty[vs]);
         }
         __syncwarp();
+        return true;
       };
-      bool ok = mbar_wait_warp(res_full, 0, abort_flag) &&
-                mbar_wait_warp(&k_full[0], 0, abort_flag) &&
-                mbar_wait_warp(&v_full[0], 0, abort_flag);
+      bool ok = mbar_wait_warp(res_full, 0, abort_flag);
       if (ok) {
         tc_fence_after();
-        issue_s(0);
-        issue_dp(0);
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int jn = j + 1;
-        const bool more = jn < n;
-        if (more) {
-          // K(j+1) and V(j+1) (both long loaded, as a rule) before S(j+1),
-          // so only the wait for the elementwise warps sits between the two
-          if (!mbar_wait_warp(&k_full[jn % KST], (jn / KST) & 1, abort_flag)) break;
-          if (!mbar_wait_warp(&v_full[jn % VST], (jn / VST) & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_s(jn);
-          if (!mbar_wait_warp(d_free, j & 1, abort_flag)) break;
-          tc_fence_after();
-          issue_dp(jn);
+        if (elect_one()) {
+          bwd_dq_copy_res<D>(tm + kBwdDqColQ, d_q);
+          bwd_dq_copy_res<D>(tm + kBwdDqColDo, d_do);
         }
-        if (!mbar_wait_warp(&p_full[j & 1], (j >> 1) & 1, abort_flag)) break;
+        __syncwarp();
+        ok = issue_s(0) && issue_dp(0);
+      }
+      if (ok && n > 1) ok = mbar_wait_warp(s_free, 0, abort_flag) && issue_s(1);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!mbar_wait_warp(ds_full, j & 1, abort_flag)) break;
         tc_fence_after();
         const uint32_t koff = (static_cast<uint32_t>(j % KST) * C::kBlockBytes) >> 4;
         if (elect_one()) {
-          if (j > 0) bwd_dq_issue_acc<D, true>(tm, tm + bwd_dq_s_col(j), d_kmn + koff);
-          else bwd_dq_issue_acc<D, false>(tm, tm + bwd_dq_s_col(j), d_kmn + koff);
-          umma_commit(&k_empty[j % KST]);
-          if (!more) umma_commit(acc_full);
+          if (j > 0) bwd_dq_issue_acc<D, true>(tm, tm + kBwdDqColDp, d_kmn + koff);
+          else bwd_dq_issue_acc<D, false>(tm, tm + kBwdDqColDp, d_kmn + koff);
+          umma_commit(&k_empty[j % KST]);    // S(j) and acc(j) were K(j)'s readers
+          if (j == n - 1) umma_commit(acc_full);
         }
         __syncwarp();
+        if (j + 1 < n && !issue_dp(j + 1)) break;
+        if (j + 2 < n && !(mbar_wait_warp(s_free, (j + 1) & 1, abort_flag) && issue_s(j + 2))) break;
       }
       if (elect_one()) umma_commit(mma_done);
       __syncwarp();
@@ -258,94 +280,99 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else {
     // ------------------------------------------------------------ elementwise
     const int ks = warp - 2;
-    const int half = ks >> 2;                           // key columns [64 half, 64 half + 64)
+    const int cg = ks >> 2;                             // key columns [32 cg, 32 cg + 32)
     const int sub = warp & 3;                           // TMEM lane quarter
     const int r = sub * 32 + lane;                      // query row of the block
     const int my_row = item.q0 + r;
     if (!skip) {
       const uint32_t lane_off = static_cast<uint32_t>(sub * 32) << 16;
-      const float sl2 = p.scale_log2;
+      const uint32_t t_s = tmem + lane_off + kBwdDqColS + cg * 32;
+      const uint32_t t_dp = tmem + lane_off + kBwdDqColDp + cg * 32;
+      const float2 sl2v = make_float2(p.scale_log2, p.scale_log2);
       const float row_nl2 = p.neg_lse2[my_row];         // -LSE in log2 units
+      const float2 nl = make_float2(row_nl2, row_nl2);
       const float row_nd = p.neg_delta[my_row];         // -D
+      const float2 nd = make_float2(row_nd, row_nd);
       bool done = true;
       for (int j = 0; j < n; ++j) {
         if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
-        const uint32_t t_s = tmem + lane_off + bwd_dq_s_col(j) + half * 64;
-        const uint32_t t_dp = tmem + lane_off + kBwdDqDpCol + half * 64;
-        uint32_t sr[64], dr[64];
-        STA_TMEM_LD32(t_s, (sr + 0));
-        STA_TMEM_LD32(t_s + 32, (sr + 32));
-        STA_TMEM_LD32(t_dp, (dr + 0));
-        STA_TMEM_LD32(t_dp + 32, (dr + 32));
+        uint32_t sr[32];
+        STA_TMEM_LD32(t_s, sr);
         tmem_wait_ld();
-        // dP's columns may take the next block's dP now
+        // S's columns may take the next block's S now
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(d_free);
+        if (lane == 0) mbar_arrive(s_free);
         // the text key block: keys >= text_len are padding
-        int hi = 64;
-        if (j >= nvid) hi = p.text_len - ((j - nvid) * 128 + half * 64);
-        uint32_t pk[32];
-        // dS = P (dP - D), P = exp2(S sl2 - lse2), two columns at a time
-        // (packed f32x2 FMA / ADD / MUL; a fixed share of the exponentials on
-        // the FMA pipe), packed to bf16 as they come
-        auto elementwise = [&](auto with_mask) {
-          const float2 sl2v = make_float2(sl2, sl2);
-          const float2 nl = make_float2(row_nl2, row_nl2);
-          const float2 nd = make_float2(row_nd, row_nd);
+        int hi = 32;
+        if (j >= nvid) hi = p.text_len - ((j - nvid) * 128 + cg * 32);
+        // P = exp2(S sl2 - lse2), two columns at a time (packed f32x2 FMA; a
+        // fixed share of the exponentials on the FMA pipe)
+        float2 pr[16];
+        auto exps = [&](auto with_mask) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
+          for (int e = 0; e < 16; ++e) {
             const int c = 2 * e;
             const float2 x = __ffma2_rn(
                 make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sl2v, nl);
-            float2 pr;
+            float2 pe;
             if (exp2_on_fma(e)) {   // resolved at compile time (unrolled)
-              pr = exp2_fma2(x);
+              pe = exp2_fma2(x);
             } else {
-              pr = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
             }
             if constexpr (decltype(with_mask)::value) {
-              if (c >= hi) pr.x = 0.f;
-              if (c + 1 >= hi) pr.y = 0.f;
+              if (c >= hi) pe.x = 0.f;
+              if (c + 1 >= hi) pe.y = 0.f;
             }
-            const float2 ds = __fmul2_rn(
-                pr, __fadd2_rn(make_float2(__uint_as_float(dr[c]), __uint_as_float(dr[c + 1])), nd));
-            pk[e] = pack_bf16x2(ds.x, ds.y);
+            pr[e] = pe;
           }
         };
-        if (hi < 64) {
-          elementwise(std::true_type{});
+        if (hi < 32) {
+          exps(std::true_type{});
         } else {
-          elementwise(std::false_type{});
+          exps(std::false_type{});
         }
-        // packed dS over the first 32 of this warp's own 64 columns of S(j)
-        STA_TMEM_ST32(t_s, pk);
+        // dS = P (dP - D), packed to bf16 over the first 16 of this warp's own
+        // 32 columns of dP(j)
+        if (!mbar_wait_warp(dp_full, j & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        uint32_t dr[32], pk[16];
+        STA_TMEM_LD32(t_dp, dr);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float2 ds = __fmul2_rn(
+              pr[e], __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]),
+                                            __uint_as_float(dr[2 * e + 1])), nd));
+          pk[e] = pack_bf16x2(ds.x, ds.y);
+        }
+        STA_TMEM_ST16(t_dp, pk);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&p_full[j & 1]);
+        if (lane == 0) mbar_arrive(ds_full);
       }
       if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
         tc_fence_after();
-        constexpr int kHalfCols = D / 2;
-        const uint32_t t_acc = tmem + lane_off + half * kHalfCols;
+        // each warp writes D / 4 columns of its rows of dQ
+        constexpr int kQCols = D / 4;
+        const uint32_t t_acc = tmem + lane_off + cg * kQCols;
         uint4* dst = reinterpret_cast<uint4*>(p.out_a + static_cast<size_t>(my_row) * D +
-                                              half * kHalfCols);
+                                              cg * kQCols);
 #pragma unroll
-        for (int cc = 0; cc < kHalfCols / 32; ++cc) {
-          uint32_t o[32];
-          STA_TMEM_LD32(t_acc + cc * 32, o);
+        for (int cc = 0; cc < kQCols / 16; ++cc) {
+          uint32_t o[16];
+          STA_TMEM_LD16(t_acc + cc * 16, o);
           tmem_wait_ld();
-          uint32_t pk2[16];
+          uint32_t pk2[8];
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
+          for (int e = 0; e < 8; ++e)
             pk2[e] = pack_bf16x2(__uint_as_float(o[2 * e]) * p.scale,
                                  __uint_as_float(o[2 * e + 1]) * p.scale);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[cc * 4 + v4] = make_uint4(pk2[4 * v4], pk2[4 * v4 + 1], pk2[4 * v4 + 2],
-                                          pk2[4 * v4 + 3]);
+          dst[cc * 2] = make_uint4(pk2[0], pk2[1], pk2[2], pk2[3]);
+          dst[cc * 2 + 1] = make_uint4(pk2[4], pk2[5], pk2[6], pk2[7]);
         }
       }
     }

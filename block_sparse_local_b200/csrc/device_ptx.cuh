@@ -146,6 +146,11 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
   return __all_sync(0xffffffffu, ok);
 }
 
+// Prefetch the global line holding `ptr` into L1.
+__device__ __forceinline__ void prefetch_l1(const void* ptr) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(reinterpret_cast<uint64_t>(ptr)));
+}
+
 // ---------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map))
@@ -387,6 +392,14 @@ __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
+// Copy a 128-row x 256-bit matrix from shared memory (described by a matrix
+// descriptor, as for an MMA operand) into TMEM lanes 0-127, 8 columns from
+// taddr.  Runs in issue order with the thread's tcgen05.mma.
+__device__ __forceinline__ void tmem_cp_128x256b(uint32_t taddr, uint64_t s_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.128x256b [%0], %1;" ::"r"(taddr), "l"(s_desc)
+               : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -446,6 +459,25 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
       "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), \
       "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), \
       "r"(r[30]), "r"(r[31])                                                   \
+      : "memory")
+
+// 32 lanes x 16 columns of 32-bit from TMEM, one row (lane) per thread.
+#define STA_TMEM_LD16(taddr, r)                                                \
+  asm volatile(                                                                \
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "                                \
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"        \
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),           \
+        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),           \
+        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),      \
+        "=r"(r[15])                                                            \
+      : "r"(taddr))
+
+#define STA_TMEM_ST8(taddr, r)                                                 \
+  asm volatile(                                                                \
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], "                           \
+      "{%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr),                               \
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),       \
+      "r"(r[6]), "r"(r[7])                                                     \
       : "memory")
 
 #define STA_TMEM_ST16(taddr, r)                                                \
@@ -561,8 +593,13 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 #define STA_EXP2_FMA_PAIRS 2
 #endif
 constexpr int kExp2FmaPairs = STA_EXP2_FMA_PAIRS;
+// Whether column pair `pair` takes exp2_fma2 when kOf8 of every 8 pairs do.
+template <int kOf8>
+__host__ __device__ constexpr bool exp2_on_fma_of(int pair) {
+  return ((pair * kOf8) / 8) != (((pair + 1) * kOf8) / 8);
+}
 __host__ __device__ constexpr bool exp2_on_fma(int pair) {
-  return ((pair * kExp2FmaPairs) / 8) != (((pair + 1) * kExp2FmaPairs) / 8);
+  return exp2_on_fma_of<kExp2FmaPairs>(pair);
 }
 
 // max(a, b, c) in one instruction (three-input max.f32 of sm_100).

@@ -1077,7 +1077,7 @@ template <int D, bool kDKV>
 sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const CUtensorMap& mdo, const sta::BwdParams& prm, int num_items,
                       cudaStream_t st) {
-  // dK/dV: attn_bwd_dkv_kernel (64-row units); dQ: attn_bwd_dq_kernel (K and V
+  // dK/dV: attn_bwd_dkv_kernel (whole streamed blocks); dQ: attn_bwd_dq_kernel (K and V
   // in separate rings, next block's scores during this block's elementwise work)
   constexpr int smem = kDKV ? sta::BwdCfg<D>::kSmemBytes : sta::BwdDqCfg<D>::kSmemBytes;
   static bool attr_set[64] = {};
@@ -1094,9 +1094,9 @@ sta_status launch_bwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
     attr_set[dev] = true;
   }
   if constexpr (kDKV)
-    sta::attn_bwd_dkv_kernel<D><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    sta::attn_bwd_dkv_kernel<D><<<num_items, sta::kDkvThreads, smem, st>>>(mq, mk, mv, mdo, prm);
   else
-    sta::attn_bwd_dq_kernel<D><<<num_items, sta::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, prm);
+    sta::attn_bwd_dq_kernel<D><<<num_items, sta::kDqThreads, smem, st>>>(mq, mk, mv, mdo, prm);
   STA_CUDA_TRY(cudaGetLastError());
   return STA_OK;
 }
