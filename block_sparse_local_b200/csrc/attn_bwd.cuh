@@ -9,7 +9,8 @@
 // This file: the preprocessing (D and the log2-domain LSE), the transposed
 // tile lists, and the dK/dV kernel, one 128-row key block per CTA: resident
 // K, V; streams the query blocks whose windows hold that key tile
-// (transposed tile lists): Q in a ring of three stages, dO in a ring of two.
+// (transposed tile lists): Q in a ring of three stages, dO in a ring of two
+// (with the block's -D, 512 bytes, next to the ring).
 // The dQ kernel is in attn_bwd_dq.cuh.
 // Every MMA has N = 128 (the whole streamed block): an MMA with N = 64
 // costs the tensor cores as long as one with N = 128.  TMEM: dV and dK
@@ -76,7 +77,8 @@ struct BwdCfg {
   static constexpr int kResV = kResK + kBlockBytes;
   static constexpr int kQRing = kResV + kBlockBytes;
   static constexpr int kDoRing = kQRing + kQStages * kBlockBytes;
-  static constexpr int kBarOff = kDoRing + kDoStages * kBlockBytes;
+  static constexpr int kDVec = kDoRing + kDoStages * kBlockBytes;   // -D of each dO stage
+  static constexpr int kBarOff = kDVec + kDoStages * 512;
   static constexpr int kSmemBytes = kBarOff + 256 + 1024;   // + 1024-byte alignment
   static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
@@ -284,17 +286,22 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
           *abort_flag = 1;
           break;
         }
-        if (pn == 0) mbar_arrive_expect_tx(&fullb[st], C::kBlockBytes);
+        if (pn == 0) mbar_arrive_expect_tx(&fullb[st], C::kBlockBytes + (is_do ? 512 : 0));
         tma_load_2d_hint(ring + st * C::kBlockBytes + pn * C::kPanelBytes, mstr, &fullb[st],
                          pn * 64, row, pol);
-        // the elementwise warps read this block's -lse2 and -D with plain
-        // loads: bring their 2 x 4 lines into L1 ahead of them
+        if (is_do && pn == 0) {
+          // the block's -D (128 floats) next to the dO ring
+          asm volatile(
+              "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+              "512, [%2];" ::"r"(smem_u32(smem + C::kDVec + st * 512)),
+              "l"(reinterpret_cast<uint64_t>(p.neg_delta + row)), "r"(smem_u32(&fullb[st]))
+              : "memory");
+        }
+        // the elementwise warps read this block's -lse2 with plain loads:
+        // bring its 4 lines into L1 ahead of them
         if (lane == 0) {
 #pragma unroll
-          for (int l = 0; l < 4; ++l) {
-            prefetch_l1(p.neg_lse2 + row + 32 * l);
-            prefetch_l1(p.neg_delta + row + 32 * l);
-          }
+          for (int l = 0; l < 4; ++l) prefetch_l1(p.neg_lse2 + row + 32 * l);
         }
       }
       __syncwarp((1u << kLanes) - 1u);
@@ -400,11 +407,12 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       const bool masked = !__all_sync(0xffffffffu, row_valid);
       bool done = true;
       for (int j = 0; j < n; ++j) {
-        // -lse2 and -D of this warp's 32 streamed rows (the same address in
-        // every lane: one L1 transaction per load)
+        // -lse2 of this warp's 32 streamed rows (the same address in every
+        // lane: one L1 transaction per load); -D from the dO stage
         const int q_row = stream_row(j) + cg * 32;
         const float4* nl4p = reinterpret_cast<const float4*>(p.neg_lse2 + q_row);
-        const float4* nd4p = reinterpret_cast<const float4*>(p.neg_delta + q_row);
+        const float4* nd4p =
+            reinterpret_cast<const float4*>(smem + C::kDVec + (j % OS) * 512) + cg * 8;
         float4 nl4v[8];
 #pragma unroll
         for (int e4 = 0; e4 < 8; ++e4) nl4v[e4] = __ldg(nl4p + e4);
@@ -441,8 +449,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
             pk_p[e] = pack_bf16x2(pe.x, pe.y);
           }
         }
-        // dS = P (dP - D)
+        // dS = P (dP - D); -D landed with dO_j
         if (!mbar_wait_warp(dp_full, j & 1, abort_flag)) { done = false; break; }
+        if (!mbar_wait_warp(&do_full[j % OS], (j / OS) & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
         // (dP^T in two halves of 16 columns, to stay within the registers of
         // 18 warps)
@@ -454,7 +463,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 nd4 = __ldg(nd4p + hf * 4 + e4);
+            const float4 nd4 = nd4p[hf * 4 + e4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int c = 2 * e4 + h2;     // column pair within the half
