@@ -9,24 +9,27 @@
 // This file: the preprocessing (D and the log2-domain LSE), the transposed
 // tile lists, and the dK/dV kernel, one 128-row key block per CTA: resident
 // K, V; streams the query blocks whose windows hold that key tile
-// (transposed tile lists): Q in a ring of three stages, dO in a ring of two
-// (with the block's -D, 512 bytes, next to the ring).
-// The dQ kernel is in attn_bwd_dq.cuh.
+// (transposed tile lists), each pipeline stage holding one Q block, its dO
+// block and its -D.  The dQ kernel is in attn_bwd_dq.cuh.
 // Every MMA has N = 128 (the whole streamed block): an MMA with N = 64
-// costs the tensor cores as long as one with N = 128.  TMEM: dV and dK
-// (fp32), chunk A = S^T of the streamed block, chunk B = dP^T and then the
-// packed P^T and dS^T.  The elementwise warps copy S^T(j) into registers
-// and release chunk A at once, so S(j+1) is computed while they work on
-// block j.  MMA order:
-//   S(0) dP(0) S(1) | dV(0) dK(0) dP(1) S(2) | dV(1) dK(1) dP(2) S(3) | ...
+// costs the tensor cores as long as one with N = 128, so 64-row units would
+// cap the kernel at about three quarters of the tensor rate.  TMEM: dV and dK
+// (fp32), chunk A = S^T of the streamed block, then its packed P^T, chunk B =
+// dP^T, then the packed dS^T.  MMA order:
+//   S(0) dP(0) | dV(0) S(1) dK(0) dP(1) | dV(1) S(2) dK(1) dP(2) | ...
+// so the elementwise warps turn S(j) into P(j) while the tensor cores run
+// dK(j-1) and dP(j), and dP(j) into dS(j) while they run dV(j) and S(j+1).
+// The per-column -LSE2 of the exponentials is loaded from global memory (L1)
+// before the wait for S(j), so its latency is off that phase's path; with
+// 16-byte broadcast loads from shared memory it sat on it, behind the score
+// MMAs' operand reads (measured: 46.6 vs 48.7 ms for the whole backward).
 // Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (scores
 // by SS tcgen05.mma, the accumulators by TS tcgen05.mma with P^T / dS^T from
 // TMEM), 2-17 elementwise: four warps per TMEM lane quarter, 32 of the 128
-// streamed rows (score columns) each.  A warp writes its packed bf16 P^T
-// and dS^T over its own 32 columns of chunk B (P^T in the first 16, dS^T in
-// the last 16), so no warp overwrites scores another warp still has to
-// read; the accumulate MMAs take two K steps of 16 rows from each warp's
-// columns.
+// streamed rows (score columns) each.  A warp writes its packed bf16 P^T /
+// dS^T into the first 16 of its own 32 columns, so no warp overwrites scores
+// another warp still has to read; the accumulate MMAs take two K steps of 16
+// rows from each warp's packed columns.
 #pragma once
 
 #include <type_traits>
@@ -71,16 +74,13 @@ struct BwdCfg {
   static constexpr int kPanels = D / 64;
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kBlockBytes = 128 * D * 2;
-  static constexpr int kQStages = 3;
-  static constexpr int kDoStages = 2;
-  static constexpr int kResK = 0;
-  static constexpr int kResV = kResK + kBlockBytes;
-  static constexpr int kQRing = kResV + kBlockBytes;
-  static constexpr int kDoRing = kQRing + kQStages * kBlockBytes;
-  static constexpr int kDVec = kDoRing + kDoStages * kBlockBytes;   // -D of each dO stage
-  static constexpr int kBarOff = kDVec + kDoStages * 512;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;   // + 1024-byte alignment
-  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+  static constexpr int kStages = 2;
+  static constexpr int kResA = 0;                                  // K (dKV) / Q (dQ)
+  static constexpr int kResB = kResA + kBlockBytes;                // V (dKV) / dO (dQ)
+  static constexpr int kStream = kResB + kBlockBytes;              // per stage: 2 blocks + -D
+  static constexpr int kStageBytes = 2 * kBlockBytes + 1024;
+  static constexpr int kBarOff = kStream + kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
 };
 
 // One warp per two rows: D[row] = sum_c dO[row,c] * O[row,c] (fp32) and the
@@ -190,22 +190,19 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                     const __grid_constant__ CUtensorMap tmap_v,
                     const __grid_constant__ CUtensorMap tmap_do, const BwdParams p) {
   using C = BwdCfg<D>;
-  constexpr int QS = C::kQStages;
-  constexpr int OS = C::kDoStages;
+  constexpr int ST = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* res_full = bars;
-  uint64_t* q_full = res_full + 1;       // [QS]
-  uint64_t* q_empty = q_full + QS;       // [QS]
-  uint64_t* do_full = q_empty + QS;      // [OS]
-  uint64_t* do_empty = do_full + OS;     // [OS]
-  uint64_t* s_full = do_empty + OS;      // S^T of the next block in chunk A
-  uint64_t* s_free = s_full + 1;         // every elementwise warp holds S^T: chunk A free
-  uint64_t* dp_full = s_free + 1;        // dP^T in chunk B
-  uint64_t* pd_full = dp_full + 1;       // packed P^T and dS^T written
-  uint64_t* acc_full = pd_full + 1;
+  uint64_t* full = res_full + 1;         // [ST]
+  uint64_t* empty = full + ST;           // [ST]
+  uint64_t* s_full = empty + ST;         // S^T of the current block in chunk A
+  uint64_t* dp_full = s_full + 1;        // dP^T in chunk B
+  uint64_t* p_full = dp_full + 1;        // packed P^T written (every elementwise warp)
+  uint64_t* ds_full = p_full + 1;        // packed dS^T written
+  uint64_t* acc_full = ds_full + 1;
   uint64_t* mma_done = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -218,7 +215,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                               item.kv_base >= 0 && item.kv_base < p.dbg_rows &&
                               item.list >= 0 && item.list < p.dbg_lists) &&
                        dbg_ok(p.counts[item.list] >= 0 && p.counts[item.list] <= p.max_k);
-  // streamed query blocks of the key block
+  // stream: key blocks of the query block (dQ) or query blocks of the key block (dK/dV)
   const int cnt = item_ok ? p.counts[item.list] : 0;
   const int* ids = p.ids + static_cast<size_t>(item_ok ? item.list : 0) * p.max_k;
   const int nvid = (cnt - p.text_sentinel) * p.tile_blocks;
@@ -233,12 +230,11 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(res_full, 1);
-    for (int i = 0; i < QS; ++i) { mbar_init(&q_full[i], 1); mbar_init(&q_empty[i], 1); }
-    for (int i = 0; i < OS; ++i) { mbar_init(&do_full[i], 1); mbar_init(&do_empty[i], 1); }
+    for (int i = 0; i < ST; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
     mbar_init(s_full, 1);
-    mbar_init(s_free, kDkvEwWarps);
     mbar_init(dp_full, 1);
-    mbar_init(pd_full, kDkvEwWarps);
+    mbar_init(p_full, kDkvEwWarps);
+    mbar_init(ds_full, kDkvEwWarps);
     mbar_init(acc_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = (error_raised() || n <= 0) ? 1 : 0;
@@ -256,130 +252,134 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const bool skip = *abort_flag != 0;
+  const uint32_t s_res_a = smem_u32(smem + C::kResA);
+  const uint32_t s_res_b = smem_u32(smem + C::kResB);
+  const uint32_t s_stream = smem_u32(smem + C::kStream);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // A thread's TMA loads complete one after another, so every operand
     // panel has its own lane: lanes 0 .. kPanels-1 the panels of resident K
     // and of the streamed Q blocks, lanes kPanels .. 2 kPanels-1 those of
-    // resident V and of the streamed dO blocks.  The first lane of each
-    // operand posts the expected bytes.
+    // resident V and of the streamed dO blocks, lane 2 kPanels the 512-byte
+    // -D copies.  Lane 0 posts the expected bytes of every stage.
     constexpr int kPanels = C::kPanels;
-    constexpr int kLanes = 2 * kPanels;
+    constexpr int kLanes = 2 * kPanels + 1;
     if (lane < kLanes && !skip) {
       const uint64_t pol = policy_evict_last();
-      const bool is_do = lane >= kPanels;
+      const int row0 = item.q0;   // the resident block
+      const bool is_b = lane >= kPanels && lane < 2 * kPanels;
+      const bool is_vec = lane == 2 * kPanels;
       const int pn = lane % kPanels;
       if (lane == 0) mbar_arrive_expect_tx(res_full, 2 * C::kBlockBytes);
-      tma_load_2d_hint(smem + (is_do ? C::kResV : C::kResK) + pn * C::kPanelBytes,
-                       is_do ? &tmap_v : &tmap_k, res_full, pn * 64, item.q0, pol);
-      const CUtensorMap* mstr = is_do ? &tmap_do : &tmap_q;
-      const int ns = is_do ? OS : QS;
-      uint64_t* fullb = is_do ? do_full : q_full;
-      uint64_t* emptyb = is_do ? do_empty : q_empty;
-      uint8_t* ring = smem + (is_do ? C::kDoRing : C::kQRing);
+      if (!is_vec) {
+        const CUtensorMap* mres = is_b ? &tmap_v : &tmap_k;
+        tma_load_2d_hint(smem + (is_b ? C::kResB : C::kResA) + pn * C::kPanelBytes, mres,
+                         res_full, pn * 64, row0, pol);
+      }
+      const CUtensorMap* mstr = is_b ? &tmap_do : &tmap_q;
       for (int j = 0; j < n; ++j) {
-        const int st = j % ns;
-        if (j >= ns && !mbar_wait(&emptyb[st], ((j / ns) - 1) & 1, abort_flag)) break;
+        const int st = j % ST;
+        if (j >= ST && !mbar_wait(&empty[st], ((j / ST) - 1) & 1, abort_flag)) break;
         const int row = stream_row(j);
         if (!dbg_ok(row >= 0 && row + 128 <= p.dbg_rows)) {
           *abort_flag = 1;
           break;
         }
-        if (pn == 0) mbar_arrive_expect_tx(&fullb[st], C::kBlockBytes + (is_do ? 512 : 0));
-        tma_load_2d_hint(ring + st * C::kBlockBytes + pn * C::kPanelBytes, mstr, &fullb[st],
-                         pn * 64, row, pol);
-        if (is_do && pn == 0) {
-          // the block's -D (128 floats) next to the dO ring
+        uint8_t* base = smem + C::kStream + st * C::kStageBytes;
+        if (lane == 0) mbar_arrive_expect_tx(&full[st], 2 * C::kBlockBytes + 512);
+        if (!is_vec) {
+          tma_load_2d_hint(base + (is_b ? C::kBlockBytes : 0) + pn * C::kPanelBytes, mstr,
+                           &full[st], pn * 64, row, pol);
+        } else {
+          // the streamed query block's -D (512 bytes)
           asm volatile(
               "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
-              "512, [%2];" ::"r"(smem_u32(smem + C::kDVec + st * 512)),
-              "l"(reinterpret_cast<uint64_t>(p.neg_delta + row)), "r"(smem_u32(&fullb[st]))
+              "512, [%2];" ::"r"(smem_u32(base + 2 * C::kBlockBytes)),
+              "l"(reinterpret_cast<uint64_t>(p.neg_delta + row)), "r"(smem_u32(&full[st]))
               : "memory");
-        }
-        // the elementwise warps read this block's -lse2 with plain loads:
-        // bring its 4 lines into L1 ahead of them
-        if (lane == 0) {
-#pragma unroll
-          for (int l = 0; l < 4; ++l) prefetch_l1(p.neg_lse2 + row + 32 * l);
         }
       }
       __syncwarp((1u << kLanes) - 1u);
       // Leave no copy in flight: wait for the last load of every stage.
       if (lane == 0) {
         mbar_wait_drain(res_full, 0);
-        for (int st = 0; st < QS && st < n; ++st) {
-          const int last = st + ((n - 1 - st) / QS) * QS;
-          mbar_wait_drain(&q_full[st], (last / QS) & 1);
-        }
-        for (int st = 0; st < OS && st < n; ++st) {
-          const int last = st + ((n - 1 - st) / OS) * OS;
-          mbar_wait_drain(&do_full[st], (last / OS) & 1);
+        for (int st = 0; st < ST && st < n; ++st) {
+          const int last = st + ((n - 1 - st) / ST) * ST;
+          mbar_wait_drain(&full[st], (last / ST) & 1);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Whole warp waits, one elected lane (always the same) issues; every MMA
-    // operand is warp-uniform and every accumulate flag a constant.  S(j+2)
-    // overwrites chunk A once every elementwise warp holds S(j+1) in
-    // registers; dP(j+1) overwrites chunk B after dV(j) and dK(j), the last
-    // readers of P(j) and dS(j): tcgen05 MMAs of one thread execute in issue
-    // order.
+    // operand is warp-uniform and every accumulate flag a constant.  S(j+1)
+    // overwrites chunk A after dV(j), the last reader of P(j), and dP(j+1)
+    // chunk B after dK(j), the last reader of dS(j): tcgen05 MMAs of one
+    // thread execute in issue order.
     if (!skip) {
       const uint32_t tm = warp_uniform(tmem);
-      const uint64_t d_res_k = sdesc_sw128(warp_uniform(smem_u32(smem + C::kResK)), 16, 1024);
-      const uint64_t d_res_v = sdesc_sw128(warp_uniform(smem_u32(smem + C::kResV)), 16, 1024);
-      const uint32_t s_q = warp_uniform(smem_u32(smem + C::kQRing));
-      const uint32_t s_do = warp_uniform(smem_u32(smem + C::kDoRing));
-      const uint64_t d_q_k = sdesc_sw128(s_q, 16, 1024);
-      const uint64_t d_q_mn = sdesc_sw128(s_q, C::kPanelBytes, 1024);
-      const uint64_t d_do_k = sdesc_sw128(s_do, 16, 1024);
-      const uint64_t d_do_mn = sdesc_sw128(s_do, C::kPanelBytes, 1024);
-      auto q_off = [](int j) { return static_cast<uint32_t>((j % QS) * C::kBlockBytes) >> 4; };
-      auto do_off = [](int j) { return static_cast<uint32_t>((j % OS) * C::kBlockBytes) >> 4; };
-      // S(j) = K Q_j^T into chunk A once Q_j has landed
-      auto issue_s = [&](int j) -> bool {
-        if (!mbar_wait_warp(&q_full[j % QS], (j / QS) & 1, abort_flag)) return false;
-        tc_fence_after();
-        if (elect_one()) {
-          bwd_issue_scores<D>(tm + kDkvColA, d_res_k, d_q_k + q_off(j));
-          umma_commit(s_full);
-        }
-        __syncwarp();
-        return true;
+      const uint64_t d_res_a = sdesc_sw128(warp_uniform(s_res_a), 16, 1024);
+      const uint64_t d_res_b = sdesc_sw128(warp_uniform(s_res_b), 16, 1024);
+      const uint64_t d_str_k = sdesc_sw128(warp_uniform(s_stream), 16, 1024);
+      const uint64_t d_str_mn = sdesc_sw128(warp_uniform(s_stream), C::kPanelBytes, 1024);
+      // descriptor offsets of a stage's first streamed block (Q or K) and of
+      // its second (dO or V)
+      auto stage_off = [](int j) {
+        return static_cast<uint32_t>((j % ST) * C::kStageBytes) >> 4;
       };
-      // dP(j) = V dO_j^T into chunk B once dO_j has landed
-      auto issue_dp = [&](int j) -> bool {
-        if (!mbar_wait_warp(&do_full[j % OS], (j / OS) & 1, abort_flag)) return false;
+      constexpr uint32_t kSecond = C::kBlockBytes >> 4;
+      bool ok = mbar_wait_warp(res_full, 0, abort_flag) && mbar_wait_warp(&full[0], 0, abort_flag);
+      if (ok) {
         tc_fence_after();
         if (elect_one()) {
-          bwd_issue_scores<D>(tm + kDkvColB, d_res_v, d_do_k + do_off(j));
+          bwd_issue_scores<D>(tm + kDkvColA, d_res_a, d_str_k);              // S^T = K Q^T
+          umma_commit(s_full);
+          bwd_issue_scores<D>(tm + kDkvColB, d_res_b, d_str_k + kSecond);    // dP^T = V dO^T
           umma_commit(dp_full);
         }
         __syncwarp();
-        return true;
-      };
-      bool ok = mbar_wait_warp(res_full, 0, abort_flag) && issue_s(0) && issue_dp(0);
-      if (ok && n > 1) ok = mbar_wait_warp(s_free, 0, abort_flag) && issue_s(1);
+      }
       for (int j = 0; ok && j < n; ++j) {
-        if (!mbar_wait_warp(pd_full, j & 1, abort_flag)) break;
+        const uint32_t so = stage_off(j);
+        const bool more = j + 1 < n;
+        if (!mbar_wait_warp(p_full, j & 1, abort_flag)) break;
         tc_fence_after();
         if (elect_one()) {
           if (j > 0) {
-            bwd_issue_acc<D, true>(tm, tm + kDkvColB, d_do_mn + do_off(j));           // dV += P^T dO
-            bwd_issue_acc<D, true>(tm + D, tm + kDkvColB + 16, d_q_mn + q_off(j));    // dK += dS^T Q
+            bwd_issue_acc<D, true>(tm, tm + kDkvColA, d_str_mn + so + kSecond);    // dV += P^T dO
           } else {
-            bwd_issue_acc<D, false>(tm, tm + kDkvColB, d_do_mn + do_off(j));
-            bwd_issue_acc<D, false>(tm + D, tm + kDkvColB + 16, d_q_mn + q_off(j));
+            bwd_issue_acc<D, false>(tm, tm + kDkvColA, d_str_mn + so + kSecond);
           }
-          umma_commit(&do_empty[j % OS]);   // dP(j) and dV(j) were the readers of dO_j
-          umma_commit(&q_empty[j % QS]);    // S(j) and dK(j) those of Q_j
-          if (j == n - 1) umma_commit(acc_full);
         }
         __syncwarp();
-        if (j + 1 < n && !issue_dp(j + 1)) break;
-        if (j + 2 < n && !(mbar_wait_warp(s_free, (j + 1) & 1, abort_flag) && issue_s(j + 2))) break;
+        if (more) {
+          const int jn = j + 1;
+          if (!mbar_wait_warp(&full[jn % ST], (jn / ST) & 1, abort_flag)) break;
+          tc_fence_after();
+          if (elect_one()) {
+            bwd_issue_scores<D>(tm + kDkvColA, d_res_a, d_str_k + stage_off(jn));
+            umma_commit(s_full);
+          }
+          __syncwarp();
+        }
+        if (!mbar_wait_warp(ds_full, j & 1, abort_flag)) break;
+        tc_fence_after();
+        if (elect_one()) {
+          if (j > 0) {
+            bwd_issue_acc<D, true>(tm + D, tm + kDkvColB, d_str_mn + so);           // dK += dS^T Q
+          } else {
+            bwd_issue_acc<D, false>(tm + D, tm + kDkvColB, d_str_mn + so);
+          }
+          umma_commit(&empty[j % ST]);   // every reader of the stage has been issued
+          if (more) {
+            bwd_issue_scores<D>(tm + kDkvColB, d_res_b, d_str_k + stage_off(j + 1) + kSecond);
+            umma_commit(dp_full);
+          } else {
+            umma_commit(acc_full);
+          }
+        }
+        __syncwarp();
       }
       if (elect_one()) umma_commit(mma_done);
       __syncwarp();
@@ -407,81 +407,81 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       const bool masked = !__all_sync(0xffffffffu, row_valid);
       bool done = true;
       for (int j = 0; j < n; ++j) {
-        // -lse2 of this warp's 32 streamed rows (the same address in every
-        // lane: one L1 transaction per load); -D from the dO stage
-        const int q_row = stream_row(j) + cg * 32;
-        const float4* nl4p = reinterpret_cast<const float4*>(p.neg_lse2 + q_row);
-        const float4* nd4p =
-            reinterpret_cast<const float4*>(smem + C::kDVec + (j % OS) * 512) + cg * 8;
+        const int st = j % ST;
+        // -lse2 of this warp's 32 streamed rows from global memory (the same
+        // address in every lane), loaded before the wait for S(j)
         float4 nl4v[8];
+        {
+          const float4* g = reinterpret_cast<const float4*>(p.neg_lse2 + stream_row(j) + cg * 32);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) nl4v[e4] = __ldg(nl4p + e4);
-        if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
-        tc_fence_after();
-        uint32_t sr[32];
-        STA_TMEM_LD32(t_a, sr);
-        tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(s_free);
-        // P = exp2(S sl2 - lse2), two columns at a time (packed f32x2 FMA; a
-        // fixed share of the exponentials on the FMA pipe), kept in fp32 for
-        // dS and packed to bf16 as they come
-        float2 pr[16];
-        uint32_t pk_p[16];
-#pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 nl4 = nl4v[e4];
-#pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int e = 2 * e4 + h2;       // column pair
-            const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
-            const float2 x = __ffma2_rn(
-                make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2v, nl);
-            float2 pe;
-            if (exp2_on_fma_of<kDkvExp2FmaPairs>(e)) {   // resolved at compile time
-              pe = exp2_fma2(x);
-            } else {
-              pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
-            }
-            if (masked && !row_valid) pe = make_float2(0.f, 0.f);
-            pr[e] = pe;
-            pk_p[e] = pack_bf16x2(pe.x, pe.y);
-          }
+          for (int e4 = 0; e4 < 8; ++e4) nl4v[e4] = __ldg(g + e4);
         }
-        // dS = P (dP - D); -D landed with dO_j
-        if (!mbar_wait_warp(dp_full, j & 1, abort_flag)) { done = false; break; }
-        if (!mbar_wait_warp(&do_full[j % OS], (j / OS) & 1, abort_flag)) { done = false; break; }
+        if (!mbar_wait_warp(s_full, j & 1, abort_flag)) { done = false; break; }
+        if (!mbar_wait_warp(&full[st], (j / ST) & 1, abort_flag)) { done = false; break; }
         tc_fence_after();
-        // (dP^T in two halves of 16 columns, to stay within the registers of
-        // 18 warps)
-        uint32_t pk_ds[16];
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t dr[16];
-          STA_TMEM_LD16(t_b + hf * 16, dr);
+        // -D of this warp's 32 streamed rows, 16-byte aligned in the stage
+        const float4* nd4p = reinterpret_cast<const float4*>(
+            smem + C::kStream + st * C::kStageBytes + 2 * C::kBlockBytes) + cg * 8;
+        // P = exp2(S sl2 - lse2), two columns at a time (packed f32x2 FMA; a
+        // fixed share of the exponentials on the FMA pipe); kept in fp32 for
+        // dS and packed to bf16 as P^T over the first 16 of the warp's columns
+        float2 pr[16];
+        {
+          uint32_t sr[32], pk[16];
+          STA_TMEM_LD32(t_a, sr);
           tmem_wait_ld();
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 nd4 = nd4p[hf * 4 + e4];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 nl4 = nl4v[e4];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
-              const int c = 2 * e4 + h2;     // column pair within the half
-              const int e = hf * 8 + c;
-              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
-              const float2 ds = __fmul2_rn(
-                  pr[e], __fadd2_rn(make_float2(__uint_as_float(dr[2 * c]),
-                                                __uint_as_float(dr[2 * c + 1])), nd));
-              pk_ds[e] = pack_bf16x2(ds.x, ds.y);
+              const int e = 2 * e4 + h2;       // column pair
+              const float2 nl = h2 ? make_float2(nl4.z, nl4.w) : make_float2(nl4.x, nl4.y);
+              const float2 x = __ffma2_rn(
+                  make_float2(__uint_as_float(sr[2 * e]), __uint_as_float(sr[2 * e + 1])), sl2v, nl);
+              float2 pe;
+              if (exp2_on_fma_of<kDkvExp2FmaPairs>(e)) {   // resolved at compile time
+                pe = exp2_fma2(x);
+              } else {
+                pe = make_float2(fast_exp2(x.x), fast_exp2(x.y));
+              }
+              if (masked && !row_valid) pe = make_float2(0.f, 0.f);
+              pr[e] = pe;
+              pk[e] = pack_bf16x2(pe.x, pe.y);
             }
           }
+          STA_TMEM_ST16(t_a, pk);     // P^T
         }
-        STA_TMEM_ST16(t_b, pk_p);          // P^T
-        STA_TMEM_ST16(t_b + 16, pk_ds);    // dS^T
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(pd_full);
+        if (lane == 0) mbar_arrive(p_full);
+        // dS = P (dP - D)
+        if (!mbar_wait_warp(dp_full, j & 1, abort_flag)) { done = false; break; }
+        tc_fence_after();
+        {
+          uint32_t dr[32], pk[16];
+          STA_TMEM_LD32(t_b, dr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 nd4 = nd4p[e4];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int e = 2 * e4 + h2;
+              const float2 nd = h2 ? make_float2(nd4.z, nd4.w) : make_float2(nd4.x, nd4.y);
+              const float2 ds = __fmul2_rn(
+                  pr[e], __fadd2_rn(make_float2(__uint_as_float(dr[2 * e]),
+                                                __uint_as_float(dr[2 * e + 1])), nd));
+              pk[e] = pack_bf16x2(ds.x, ds.y);
+            }
+          }
+          STA_TMEM_ST16(t_b, pk);     // dS^T
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_full);
       }
       if (done && mbar_wait_warp(acc_full, 0, abort_flag)) {
         tc_fence_after();
