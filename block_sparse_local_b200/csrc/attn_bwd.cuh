@@ -75,12 +75,15 @@ struct BwdCfg {
   static constexpr int kPanelBytes = 128 * 128;
   static constexpr int kBlockBytes = 128 * D * 2;
   static constexpr int kStages = 2;
-  static constexpr int kResA = 0;                                  // K (dKV) / Q (dQ)
-  static constexpr int kResB = kResA + kBlockBytes;                // V (dKV) / dO (dQ)
-  static constexpr int kStream = kResB + kBlockBytes;              // per stage: 2 blocks + -D
+  static constexpr int kResA = 0;                                  // resident K
+  static constexpr int kResB = kResA + kBlockBytes;                // resident V
+  static constexpr int kStream = kResB + kBlockBytes;              // per stage: Q, dO, -D
+  // -D takes 512 bytes; the stage stride stays a multiple of 1024 so that
+  // every 128-byte-swizzled block starts on a 1024-byte boundary
   static constexpr int kStageBytes = 2 * kBlockBytes + 1024;
   static constexpr int kBarOff = kStream + kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarOff + 256 + 1024;
+  static constexpr int kSmemBytes = kBarOff + 256 + 1024;   // + 1024-byte alignment
+  static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 };
 
 // One warp per two rows: D[row] = sum_c dO[row,c] * O[row,c] (fp32) and the

@@ -3,9 +3,9 @@
 // dQ = dS K / sqrt(d) with dS = P (dP - D), P = exp2(S log2(e)/sqrt(d) - LSE2),
 // S = Q K^T and dP = dO V^T over the key blocks of the query block's window
 // (the forward's tile lists).  One 128-row query block per CTA: Q and dO
-// resident in shared memory, K and V streamed in separate TMA rings, K in
-// three stages (released after dQ += dS K reads it) and V in two (released
-// right after the dP MMA, its only reader).
+// loaded once into shared memory and copied into TMEM, K and V streamed in
+// separate TMA rings, K in three stages (released after dQ += dS K reads it)
+// and V in two (released right after the dP MMA, its only reader).
 //
 // TMEM: the dQ accumulator in columns [0, 128); the resident Q and dO,
 // packed bf16, in [128, 192) and [192, 256) (copied from shared memory by
@@ -19,9 +19,8 @@
 // Warps: 0 TMA producer (one lane per operand panel), 1 MMA issuer (the whole
 // warp waits, one elected lane issues; warp-uniform operands, constant
 // accumulate flags), 2-17 elementwise: four warps per TMEM lane quarter, 32
-// of the 128 key columns each (the dS work of block j+1 sits on the loop
-// acc(j) -> dP(j+1) -> dS(j+1), so it is spread over as many warps as the
-// registers allow).
+// of the 128 key columns each (8 warps of 64 columns measured the same; 16
+// need fewer registers per thread).
 #pragma once
 
 #include <type_traits>
